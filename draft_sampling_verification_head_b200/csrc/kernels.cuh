@@ -1,0 +1,89 @@
+// Internal interfaces between the C-ABI layer and the kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace specdec {
+
+struct RowPartial {
+  float m;      // max of raw logits over the segment
+  float s;      // sum exp2((x - m) * k)
+  float amax;   // arg-max value
+  int32_t aidx; // arg-max index (lowest on ties)
+};
+
+struct StopInfo {
+  int32_t j;   // stop row (K = all drafts accepted, bonus from row K)
+  float mt;    // target row j softmax stats
+  float st;
+  float mz;    // draft row j softmax stats
+  float sz;
+};
+
+// ---- Markov bias, one step -------------------------------------------------
+size_t bias_tc_smem_bytes(int r, int N);
+cudaError_t launch_bias_tc(const CUtensorMap& tmW, const __nv_bfloat16* U, const int32_t* prev,
+                           float* bias, int B, int V, int r, WsHeader* hdr, uint64_t spin,
+                           cudaStream_t st);
+template <typename T>
+cudaError_t launch_bias_fma(const T* U, const T* W, const int32_t* prev, float* bias, int B, int V,
+                            int r, WsHeader* hdr, cudaStream_t st);
+
+// ---- Stand-alone verification ----------------------------------------------
+int verify_seg_len(int V);
+size_t verify_ws_bytes(int B, int K, int V);
+template <typename T, typename TD>
+cudaError_t launch_verify(const T* target, const TD* draft_logits, const int32_t* draft,
+                          int32_t* out, int32_t* tau, float* p_draft, float* q_draft, int B,
+                          int K, int V, float temperature, int greedy, uint64_t seed,
+                          uint64_t cycle, uint8_t* ws_body, WsHeader* hdr, int num_sms,
+                          cudaStream_t st, int* launches);
+
+// ---- Fused persistent draft (+ verify) ---------------------------------------
+enum CycleMode : int32_t { MODE_CYCLE = 0, MODE_DRAFT = 1 };
+
+struct CycleGeom {
+  int G;        // CTAs (one per SM at most)
+  int nc;       // 128-token chunks per CTA
+  int nchunks;  // ceil(V / 128)
+  int N;        // batch rows per group (MMA N): 16, 32 or 64
+  bool tc;      // tensor-core bias
+  size_t smem;  // dynamic shared memory bytes
+};
+
+// Decide the launch geometry; returns false (with a reason) if unsupported.
+bool cycle_geometry(int B, int K, int V, int r, int dtype, uint32_t flags, int num_sms,
+                    CycleGeom* g, const char** why);
+size_t cycle_ws_bytes(int K, const CycleGeom& g);
+
+struct CycleLaunch {
+  const void* base;
+  const void* target;
+  const void* U;
+  const void* W;
+  const int32_t* last_token;
+  int32_t* draft;
+  int32_t* out;
+  int32_t* tau;
+  float* p_draft;
+  float* q_draft;
+  float* biased_out;
+  int B, K, V, r, dtype, mode, greedy;
+  float temperature;
+  uint64_t seed, cycle, spin;
+};
+
+cudaError_t launch_cycle(const CycleLaunch& L, const CycleGeom& g, WsHeader* hdr, uint8_t* body,
+                         const CUtensorMap* tmW, const CUtensorMap* tmBase, cudaStream_t st);
+
+// ---- Tensor maps --------------------------------------------------------------
+bool make_tmap_W(CUtensorMap* m, const void* W, int r, int V);
+bool make_tmap_base(CUtensorMap* m, const void* base, int dtype, int B, int K, int V, int N);
+
+// ---- Debug ------------------------------------------------------------------------
+cudaError_t launch_debug_philox(const uint32_t* ctr, const uint32_t* key, uint32_t* out, int n,
+                                cudaStream_t st);
+cudaError_t launch_debug_curand_philox(const uint32_t* ctr, const uint32_t* key, uint32_t* out,
+                                       int n, cudaStream_t st);
+
+}  // namespace specdec

@@ -1,0 +1,150 @@
+/*
+ * specdec -- the draft-sample-and-verify step of block-parallel speculative
+ * decoding on NVIDIA B200 (sm_100a), as a C-ABI library (libspecdec.so).
+ *
+ * The step (pages: aigest.pl "DeepSeek prezentuje DSpark"; telemetr.me DFlash
+ * post; mkdocs.reaper.mx DeepSeek-V4.1-Flash "06-extensions", DSpark table):
+ *   a parallel drafter gives base logits for K block positions in one pass;
+ *   a sequential Markov head adds bias_i = U[prev] . W (rank r) before each
+ *   draft token is sampled, prev being the last committed token for i = 0 and
+ *   the previous draft token after that ("Innowacje w tworzeniu tokenów");
+ *   the target's K+1 logit rows then verify the block by rejection sampling:
+ *   the longest accepted prefix plus one extra token, with the target
+ *   distribution preserved exactly ("Jak działa spekulatywne dekodowanie").
+ *   Accept d_i iff u < min(1, p_i(d_i)/q_i(d_i)); at the first rejection emit
+ *   a draw from max(p_i - q_i, 0) normalised (p_i if that is all zero); if all
+ *   K pass, emit a bonus draw from target row K.  Greedy mode drafts arg-max
+ *   tokens and accepts while arg-max(target_i) equals d_i.  tau = accepted + 1
+ *   is the quantity in L = (T_draft + T_verify) / tau.
+ *   p = softmax(target / T), q = softmax((base + bias) / T).
+ *
+ * Random numbers: Philox4x32-10 (Salmon et al., SC'11), key = seed,
+ * counter = (position, batch row, lo32(cycle), tag | bits 32..47 of cycle << 16),
+ * word 0 mapped to [0,1) as (x >> 8) * 2^-24; tag 0 = draft draw, 1 = accept
+ * test, 2 = residual or bonus draw.  Sampling is by inverse CDF in ascending
+ * token order: the first token whose inclusive prefix mass exceeds u * total.
+ * Ties in arg-max go to the lowest index.
+ *
+ * Layouts (row-major, V contiguous, caller-owned device memory):
+ *   base        [B, K, V]    dtype        draft base logits
+ *   target      [B, K+1, V]  dtype        target logits, row K = bonus row
+ *   U           [V, r]       dtype        Markov factor, row = previous token
+ *   W           [r, V]       dtype        Markov factor
+ *   last_token  [B]          int32        last committed token
+ *   draft       [B, K]       int32        draft tokens d_i
+ *   out         [B, K+1]     int32        emitted tokens; entries >= tau are -1
+ *   tau         [B]          int32        1 .. K+1
+ *   p_draft     [B, K]       float        p_i(d_i) where the accept test ran, NaN after
+ *   q_draft     [B, K]       float        q_i(d_i)
+ *   biased_out  [B, K, V]    float        z = base + bias (optional)
+ * dtype is SPEC_BF16 (bf16 logits and factors; bias products on tcgen05
+ * tensor cores, fp32 accumulate) or SPEC_F32 (fp32 throughout).  All
+ * arithmetic after loading is fp32.  In greedy mode p_draft / q_draft are
+ * filled with NaN.
+ *
+ * Calls are asynchronous on `stream`.  Errors found on the host (bad sizes,
+ * NULL pointers, a workspace too small) are returned before anything is
+ * launched.  Errors found on the device (a token id out of range, a wait that
+ * ran past spin_limit polls) are recorded in the workspace and returned by
+ * spec_sync_status().  Every device-side wait is bounded; a kernel that gives
+ * up records SPEC_ERR_TIMEOUT and returns, leaving the outputs undefined.
+ * One workspace serves one stream at a time; calls that share a workspace
+ * must be ordered on one stream.
+ */
+#ifndef SPECDEC_H
+#define SPECDEC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st *spec_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  SPEC_OK = 0,
+  SPEC_ERR_INVALID_ARG = -1,   /* NULL pointer, size out of range, bad temperature */
+  SPEC_ERR_UNSUPPORTED = -2,   /* shape the kernels do not handle (message says which) */
+  SPEC_ERR_CUDA = -3,          /* a CUDA runtime call failed */
+  SPEC_ERR_TIMEOUT = -4,       /* a device-side wait exceeded spin_limit polls */
+  SPEC_ERR_WORKSPACE = -5,     /* workspace NULL, too small or misaligned */
+  SPEC_ERR_TOKEN_RANGE = -6    /* a token id (last_token / draft) outside [0, V) */
+} spec_status;
+
+typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
+
+/* Flags */
+#define SPEC_FLAG_FMA_BIAS 1u  /* compute the Markov bias with fp32 FMAs instead of tensor cores */
+
+typedef struct {
+  int32_t B;             /* batch rows, >= 1 */
+  int32_t K;             /* draft block length, 1 .. 64 */
+  int32_t V;             /* vocabulary, >= 1; bf16 needs V % 8 == 0, f32 V % 4 == 0 */
+  int32_t r;             /* Markov rank: 0 (no head) or 1..256; bf16 tensor-core path needs r % 64 == 0 */
+  int32_t dtype;         /* spec_dtype of base, target, U, W */
+  int32_t draft_dtype;   /* spec_verify_block: spec_dtype of draft_logits */
+  float temperature;     /* > 0 unless greedy */
+  int32_t greedy;        /* 0 = stochastic, 1 = greedy */
+  uint64_t seed;         /* Philox key */
+  uint64_t cycle;        /* Philox counter words 2..3 (advance it every cycle) */
+  uint64_t spin_limit;   /* polls before a device wait gives up; 0 = default (about 2 s) */
+  uint32_t flags;        /* SPEC_FLAG_* */
+  uint32_t reserved;
+} spec_params;
+
+/* Bytes of device workspace the calls need for these parameters on the
+ * current device (0 if the parameters are invalid).  Alignment: 256 bytes. */
+size_t spec_workspace_size(const spec_params *p);
+
+/* Zero a workspace (asynchronously on `stream`).  Required once before first
+ * use, and again after any call whose spec_sync_status was not SPEC_OK. */
+spec_status spec_workspace_init(void *workspace, size_t bytes, spec_stream_t stream);
+
+/* Markov-head bias for one draft step (section "Innowacje w tworzeniu
+ * tokenów"): bias[b, v] = sum_k U[prev[b], k] * W[k, v], fp32 accumulate.
+ * prev [B] int32 (device), bias [B, V] float (device). */
+spec_status spec_markov_bias(const spec_params *p, const void *U, const void *W,
+                             const int32_t *prev, float *bias, void *workspace,
+                             spec_stream_t stream);
+
+/* Sequential drafting: for i = 0..K-1, z = base_i + U[prev] . W, d_i drawn
+ * from softmax(z / T) (arg-max in greedy mode), prev = d_i.  One persistent
+ * launch carries all K steps.  q_draft and biased_out may be NULL. */
+spec_status spec_markov_bias_sample(const spec_params *p, const void *base, const void *U,
+                                    const void *W, const int32_t *last_token, int32_t *draft,
+                                    float *q_draft, float *biased_out, void *workspace,
+                                    spec_stream_t stream);
+
+/* Verification of given drafts against the target rows (section "Jak działa
+ * spekulatywne dekodowanie"): draft_logits [B, K, V] are the final (biased)
+ * draft logits in draft_dtype, draft [B, K] the tokens drawn from them.
+ * p_draft and q_draft may be NULL. */
+spec_status spec_verify_block(const spec_params *p, const void *target, const void *draft_logits,
+                              const int32_t *draft, int32_t *out, int32_t *tau, float *p_draft,
+                              float *q_draft, void *workspace, spec_stream_t stream);
+
+/* One whole cycle: drafting and verification fused in one persistent launch
+ * (target rows are read only up to each row's first rejection).  draft,
+ * p_draft and q_draft may be NULL. */
+spec_status spec_cycle(const spec_params *p, const void *base, const void *target, const void *U,
+                       const void *W, const int32_t *last_token, int32_t *draft, int32_t *out,
+                       int32_t *tau, float *p_draft, float *q_draft, void *workspace,
+                       spec_stream_t stream);
+
+/* Synchronise `stream` and return the device-side status recorded in the
+ * workspace by the calls issued on it (SPEC_OK if none failed). */
+spec_status spec_sync_status(const void *workspace, spec_stream_t stream);
+
+/* Human-readable name of a status code. */
+const char *spec_status_string(spec_status s);
+
+/* Number of kernel launches the last call on this thread issued. */
+int32_t spec_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

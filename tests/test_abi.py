@@ -1,0 +1,78 @@
+"""The C-ABI library loads and exports every symbol the headers declare; host
+argument checks answer before any launch (CPU only, no GPU needed)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import draft_sampling_verification_head_b200 as sd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"\b(spec_[a-z_0-9]+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    declared = _declared()
+    assert {"spec_cycle", "spec_markov_bias_sample", "spec_verify_block"} <= declared
+    lib = ctypes.CDLL(sd.LIB_PATH)
+    for name in sorted(declared):
+        assert hasattr(lib, name), name
+    assert declared == set(sd._SIGS), "binding signatures out of sync with the headers"
+
+
+def test_status_strings():
+    for code, name in [(0, "SPEC_OK"), (-1, "SPEC_ERR_INVALID_ARG"), (-4, "SPEC_ERR_TIMEOUT"),
+                       (-6, "SPEC_ERR_TOKEN_RANGE")]:
+        assert sd.status_string(code) == name
+
+
+def _p(**kw):
+    d = dict(B=4, K=4, V=1024, r=16, dtype="bf16", temperature=1.0)
+    d.update(kw)
+    return sd.Params(**d)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), sd.SPEC_ERR_INVALID_ARG),
+    (dict(K=0), sd.SPEC_ERR_INVALID_ARG),
+    (dict(r=300), sd.SPEC_ERR_INVALID_ARG),
+    (dict(temperature=0.0), sd.SPEC_ERR_INVALID_ARG),
+    (dict(V=1001), sd.SPEC_ERR_UNSUPPORTED),
+])
+def test_host_validation_before_launch(kw, code):
+    L = sd.lib()
+    p = _p(**kw).c()
+    fake = ctypes.c_void_p(0x1000)
+    rc = L.spec_cycle(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, None, None,
+                      fake, None)
+    assert rc == code
+    assert L.spec_workspace_size(ctypes.byref(p)) == 0
+
+
+def test_null_pointers_rejected():
+    L = sd.lib()
+    p = _p().c()
+    rc = L.spec_cycle(ctypes.byref(p), None, None, None, None, None, None, None, None, None, None,
+                      None, None)
+    assert rc == sd.SPEC_ERR_INVALID_ARG
+    assert L.spec_cycle(None, *([None] * 12)) == sd.SPEC_ERR_INVALID_ARG
+    assert L.spec_workspace_init(None, 0, None) == sd.SPEC_ERR_WORKSPACE
+
+
+def test_greedy_allows_zero_temperature_shape_check():
+    L = sd.lib()
+    p = _p(temperature=0.0, greedy=True, V=1001).c()
+    fake = ctypes.c_void_p(0x1000)
+    # passes the temperature rule, then fails on the vocabulary alignment rule
+    assert L.spec_cycle(ctypes.byref(p), *([fake] * 6), fake, fake, None, None, fake,
+                        None) == sd.SPEC_ERR_UNSUPPORTED

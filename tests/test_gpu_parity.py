@@ -1,0 +1,320 @@
+"""CUDA path vs the oracle, through the C-ABI (needs a B200).
+
+Bit-exact tokens and accepted lengths except decisions the oracle flags as
+within 1e-6 of a threshold (counted); probabilities within 1e-5 absolute.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+from scipy import stats
+
+import oracle
+import synth
+from oracle import exact_law as EL
+from parity import check_invariants, compare_cycle, compare_draft
+
+import draft_sampling_verification_head_b200 as sd
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    sd.lib()
+    oracle.build()
+
+
+def _dev(d):
+    return {k: v.cuda() for k, v in d.items()}
+
+
+def _np(t):
+    return t.cpu().numpy()
+
+
+def gpu_cycle(w, d, greedy=False, T=None, seed=0, cyc=0, flags=0, spin=0, dd=None):
+    T = w.temperature if T is None else T
+    p = sd.Params(B=d["base"].shape[0], K=w.K, V=w.V, r=w.r, dtype=w.dtype, temperature=T,
+                  greedy=greedy, seed=seed, cycle=cyc, flags=flags, spin_limit=spin)
+    dd = dd or _dev(d)
+    ws = sd.make_workspace(p)
+    o = sd.alloc_outputs(p)
+    sd.cycle(p, dd["base"], dd["target"], dd["U"], dd["W"], dd["last_token"], o["draft"], o["out"],
+             o["tau"], o["p_draft"], o["q_draft"], ws)
+    st = sd.sync_status(ws)
+    assert st == sd.SPEC_OK, sd.status_string(st)
+    return {k: _np(v) for k, v in o.items()}
+
+
+def orc_cycle(w, d, greedy=False, T=None, seed=0, cyc=0, b_begin=0, b_end=None):
+    T = w.temperature if T is None else T
+    P = oracle.Params(B=d["base"].shape[0], K=w.K, V=w.V, r=w.r, dtype=w.dtype, temperature=T,
+                      greedy=greedy, seed=seed, cycle=cyc)
+    return oracle.cycle(P, *(synth.to_numpy_raw(d[k]) for k in ("base", "target", "U", "W")),
+                        d["last_token"].numpy(), b_begin=b_begin, b_end=b_end)
+
+
+# ----------------------------------------------------------------------------- random stream
+
+def test_philox_bit_exact_vs_oracle_and_curand():
+    n = 1 << 16
+    g = torch.Generator().manual_seed(7)
+    ctr = torch.randint(0, 2 ** 31, (n, 4), generator=g, dtype=torch.int64)
+    ctr[: n // 4] = torch.randint(0, 64, (n // 4, 4), generator=g)  # small counters too
+    # curand takes counter words 0..1 as a 64-bit offset times four: keep word 1 below 2^30
+    ctr[:, 1] &= (1 << 30) - 1
+    key = torch.randint(0, 2 ** 31, (n, 2), generator=g, dtype=torch.int64)
+    key[:, 0] |= 1 << 31  # exercise the top bit
+    c32 = ctr.to(torch.int32).cuda()
+    k32 = key.to(torch.int32).cuda()
+    out = torch.zeros((n, 4), dtype=torch.int32, device="cuda")
+    ref = torch.zeros_like(out)
+    sd.debug_philox(c32, k32, out)
+    sd.debug_curand_philox(c32, k32, ref)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref), "kernel Philox differs from the CUDA library's Philox4_32_10"
+    got = out.cpu().numpy().view(np.uint32)
+    for i in range(0, n, 97):
+        assert list(got[i]) == oracle.philox(ctr[i].tolist(), key[i].tolist()), i
+    # full 32-bit counter words against the oracle
+    ctr2 = torch.randint(0, 2 ** 32, (4096, 4), generator=g, dtype=torch.int64)
+    out2 = torch.zeros((4096, 4), dtype=torch.int32, device="cuda")
+    sd.debug_philox(ctr2.to(torch.int32).cuda(), k32[:4096].contiguous(), out2)
+    got2 = out2.cpu().numpy().view(np.uint32)
+    for i in range(4096):
+        assert list(got2[i]) == oracle.philox(ctr2[i].tolist(), key[i].tolist()), i
+
+
+# ----------------------------------------------------------------------------- Markov bias
+
+@pytest.mark.parametrize("B,V,r,dtype,flags", [
+    (37, 1000, 256, "bf16", 0), (64, 4096, 64, "bf16", 0), (5, 2048, 128, "bf16", 0),
+    (200, 1536, 256, "bf16", 0), (37, 1000, 256, "bf16", sd.SPEC_FLAG_FMA_BIAS),
+    (9, 1024, 16, "f32", 0)])
+def test_markov_bias_vs_matmul(B, V, r, dtype, flags):
+    w = synth.Workload("mb", B=B, K=1, V=V, r=r, dtype=dtype, seed=31)
+    d = synth.make(w)
+    prev = torch.randint(0, V, (B,), generator=torch.Generator().manual_seed(3)).to(torch.int32)
+    p = sd.Params(B=B, K=1, V=V, r=r, dtype=dtype, flags=flags)
+    ws = sd.make_workspace(p)
+    bias = torch.full((B, V), float("nan"), device="cuda")
+    sd.markov_bias(p, d["U"].cuda(), d["W"].cuda(), prev.cuda(), bias, ws)
+    assert sd.sync_status(ws) == sd.SPEC_OK
+    ref = d["U"].double()[prev.long()] @ d["W"].double()
+    scale = d["U"].double().abs()[prev.long()] @ d["W"].double().abs()
+    err = (bias.cpu().double() - ref).abs()
+    assert torch.all(err <= 1e-6 * scale + 1e-9), float((err / (scale + 1e-12)).max())
+
+
+# ----------------------------------------------------------------------------- drafting only
+
+@pytest.mark.parametrize("greedy", [False, True])
+@pytest.mark.parametrize("B,K,V,r,dtype,flags", [
+    (5, 4, 1000, 64, "bf16", 0), (19, 3, 4096, 256, "bf16", 0), (6, 5, 800, 16, "f32", 0),
+    (5, 4, 1000, 64, "bf16", sd.SPEC_FLAG_FMA_BIAS)])
+def test_markov_bias_sample_vs_oracle(B, K, V, r, dtype, flags, greedy):
+    w = synth.Workload("ds", B=B, K=K, V=V, r=r, dtype=dtype, seed=41, uw_std=0.3)
+    d = synth.make(w)
+    p = sd.Params(B=B, K=K, V=V, r=r, dtype=dtype, temperature=0.9, greedy=greedy, seed=5,
+                  cycle=11, flags=flags)
+    ws = sd.make_workspace(p)
+    dd = _dev(d)
+    draft = torch.full((B, K), -7, dtype=torch.int32, device="cuda")
+    q = torch.full((B, K), -1.0, device="cuda")
+    biased = torch.zeros((B, K, V), device="cuda")
+    sd.markov_bias_sample(p, dd["base"], dd["U"], dd["W"], dd["last_token"], draft, q, biased, ws)
+    assert sd.sync_status(ws) == sd.SPEC_OK
+    P = oracle.Params(B=B, K=K, V=V, r=r, dtype=dtype, temperature=0.9, greedy=greedy, seed=5,
+                      cycle=11)
+    o = oracle.draft(P, *(synth.to_numpy_raw(d[k]) for k in ("base", "U", "W")),
+                     d["last_token"].numpy(), biased=True)
+    flagged = compare_draft({"draft": _np(draft), "q_draft": _np(q)}, o, K)
+    assert flagged <= max(1, B // 10)
+    # biased logits up to the first flagged draft (later rows depend on the draws)
+    bz = _np(biased)
+    for b in range(B):
+        fd = int(o["flag_draft"][b])
+        np.testing.assert_allclose(bz[b, :fd], o["biased"][b, :fd], rtol=0, atol=2e-5)
+    if greedy:
+        assert np.all(np.isnan(_np(q)))
+
+
+# ----------------------------------------------------------------------------- verification only
+
+@pytest.mark.parametrize("greedy", [False, True])
+@pytest.mark.parametrize("B,K,V,dtype,ddtype", [
+    (7, 4, 1000, "bf16", "bf16"), (16, 6, 20000, "bf16", "f32"), (5, 3, 512, "f32", "f32"),
+    (3, 2, 40000, "f32", "bf16")])
+def test_verify_block_vs_oracle(B, K, V, dtype, ddtype, greedy):
+    w = synth.Workload("vb", B=B, K=K, V=V, r=8, dtype=dtype, sigma=0.7, seed=51)
+    d = synth.make(w)
+    # draft logits: base perturbed, in the requested dtype; drafts drawn by the oracle
+    g = torch.Generator().manual_seed(9)
+    dl = (d["base"].float() + 0.3 * torch.randn(d["base"].shape, generator=g))
+    dl = dl.to(torch.bfloat16 if ddtype == "bf16" else torch.float32)
+    P = oracle.Params(B=B, K=K, V=V, r=0, dtype=dtype, draft_dtype=ddtype, temperature=1.2,
+                      greedy=greedy, seed=3, cycle=5)
+    drafts = oracle.draft(oracle.Params(B=B, K=K, V=V, r=0, dtype=ddtype, temperature=1.2,
+                                        greedy=greedy, seed=3, cycle=5),
+                          synth.to_numpy_raw(dl), np.zeros((V, 0), np.uint16 if ddtype == "bf16" else np.float32),
+                          np.zeros((0, V), np.uint16 if ddtype == "bf16" else np.float32),
+                          d["last_token"].numpy())["draft"]
+    o = oracle.verify(P, synth.to_numpy_raw(d["target"]), synth.to_numpy_raw(dl), drafts)
+    p = sd.Params(B=B, K=K, V=V, r=0, dtype=dtype, draft_dtype=ddtype, temperature=1.2,
+                  greedy=greedy, seed=3, cycle=5)
+    ws = sd.make_workspace(p)
+    outs = sd.alloc_outputs(p)
+    sd.verify_block(p, d["target"].cuda(), dl.cuda(), torch.from_numpy(drafts).cuda(), outs["out"],
+                    outs["tau"], outs["p_draft"], outs["q_draft"], ws)
+    assert sd.sync_status(ws) == sd.SPEC_OK
+    gpu = {k: _np(v) for k, v in outs.items()}
+    gpu["draft"] = drafts
+    o["draft"] = drafts
+    o["flag_draft"] = np.full(B, K, np.int32)
+    compare_cycle(gpu, o, K)
+    check_invariants(gpu["out"], gpu["tau"], drafts, K)
+
+
+# ----------------------------------------------------------------------------- fused cycle
+
+CASES = [
+    # name, workload, greedy, temperature
+    ("small_ragged", synth.Workload("s", B=5, K=3, V=1000, r=64, dtype="bf16", sigma=0.6, seed=61,
+                                    uw_std=0.3), False, 1.0),
+    ("small_ragged_greedy", synth.Workload("s", B=5, K=3, V=1000, r=64, dtype="bf16", sigma=0.6,
+                                           seed=61, uw_std=0.3), True, 1.0),
+    ("multi_group", synth.Workload("mg", B=70, K=4, V=2048, r=128, dtype="bf16", sigma=0.4,
+                                   seed=62, uw_std=0.2), False, 0.8),
+    ("c1", synth.WORKLOADS["c1"], False, 1.0),
+    ("c1_greedy", synth.WORKLOADS["c1"], True, 1.0),
+    ("c2_t07", synth.WORKLOADS["c2"], False, 0.7),
+    ("c2_greedy", synth.WORKLOADS["c2"], True, 0.7),
+    ("f32_no_head", synth.Workload("nh", B=9, K=5, V=3000, r=0, dtype="f32", sigma=0.5, seed=63),
+     False, 1.0),
+    ("fma_bias", synth.Workload("fb", B=6, K=4, V=5000, r=64, dtype="bf16", sigma=0.5, seed=64,
+                                uw_std=0.3), False, 1.0),
+]
+
+
+@pytest.mark.parametrize("name,w,greedy,T", CASES, ids=[c[0] for c in CASES])
+def test_cycle_vs_oracle(name, w, greedy, T):
+    d = synth.make(w)
+    flags = sd.SPEC_FLAG_FMA_BIAS if name == "fma_bias" else 0
+    total_flag = 0
+    for cyc in range(2):
+        g = gpu_cycle(w, d, greedy=greedy, T=T, seed=17, cyc=cyc, flags=flags)
+        o = orc_cycle(w, d, greedy=greedy, T=T, seed=17, cyc=cyc)
+        total_flag += compare_cycle(g, o, w.K)
+        check_invariants(g["out"], g["tau"], g["draft"], w.K)
+    assert total_flag <= max(1, d["base"].shape[0] // 10)
+
+
+def test_cycle_deterministic():
+    w = CASES[2][1]
+    d = synth.make(w)
+    a = gpu_cycle(w, d, T=0.8, seed=1)
+    b = gpu_cycle(w, d, T=0.8, seed=1)
+    for k in ("draft", "out", "tau"):
+        assert np.array_equal(a[k], b[k])
+    np.testing.assert_array_equal(a["q_draft"], b["q_draft"])
+
+
+def test_cycle_target_equals_draft_accepts_everything():
+    w = synth.Workload("eq", B=12, K=6, V=4096, r=64, dtype="bf16", uw_std=0.0, seed=65)
+    d = synth.make(w)
+    d["target"] = torch.cat([d["base"], d["base"][:, :1]], dim=1).contiguous()
+    for greedy in (False, True):
+        g = gpu_cycle(w, d, greedy=greedy)
+        assert np.all(g["tau"] == w.K + 1)
+        assert np.array_equal(g["out"][:, : w.K], g["draft"])
+
+
+@pytest.mark.parametrize("cfg,rows", [("c3", [0, 1, 2, 63]), ("c4", [0, 255]), ("c5", [0, 127])])
+def test_cycle_full_size_sampled_rows(cfg, rows):
+    """Full-size launch (the benchmark's configuration); the oracle checks
+    sampled rows one by one."""
+    w = synth.WORKLOADS[cfg]
+    d = synth.make(w)
+    g = gpu_cycle(w, d, seed=w.seed, cyc=1)
+    check_invariants(g["out"], g["tau"], g["draft"], w.K)
+    flagged = 0
+    for b in rows:
+        o = orc_cycle(w, d, seed=w.seed, cyc=1, b_begin=b, b_end=b + 1)
+        gb = {k: v[b:b + 1] for k, v in g.items()}
+        flagged += compare_cycle(gb, o, w.K, rows=[b])
+    assert flagged <= 1
+
+
+def test_exact_distribution_v8_k3():
+    """V=8, K=3: 10^6 seeded cycles (one batch row per cycle) against the
+    enumerated exact law of the emitted tokens."""
+    w = synth.WORKLOADS["c5b"]
+    d0 = synth.make(w)
+    n = 1_000_000
+    d = {"base": d0["base"].expand(n, -1, -1).contiguous(),
+         "target": d0["target"].expand(n, -1, -1).contiguous(),
+         "U": d0["U"], "W": d0["W"],
+         "last_token": d0["last_token"].expand(n).contiguous()}
+    g = gpu_cycle(w, d, seed=123, cyc=0)
+    law = EL.exact_law(synth.as_float64(d0["base"])[0], synth.as_float64(d0["target"])[0],
+                       synth.as_float64(d0["U"]), synth.as_float64(d0["W"]),
+                       int(d0["last_token"][0]), 1.0)
+    first, pair, taus = EL.cell_probs(law, w.K, w.V)
+    out, tau = g["out"], g["tau"]
+
+    def pooled(obs, p, m):
+        e = p * m
+        keep = e >= 5
+        o_ = np.append(obs[keep], obs[~keep].sum())
+        e_ = np.append(e[keep], e[~keep].sum())
+        if e_[-1] == 0:
+            o_, e_ = o_[:-1], e_[:-1]
+        return stats.chisquare(o_, e_ * o_.sum() / e_.sum()).pvalue
+
+    sel = tau >= 2
+    pv = [pooled(np.bincount(out[:, 0], minlength=w.V), first, n),
+          pooled(np.bincount(out[sel, 0] * w.V + out[sel, 1], minlength=w.V * w.V),
+                 pair.ravel() / pair.sum(), int(sel.sum())),
+          pooled(np.bincount(tau - 1, minlength=w.K + 1), taus, n)]
+    assert min(pv) > 1e-3, pv
+    acc = taus[1:].sum()
+    assert abs(sel.mean() - acc) < 4 * math.sqrt(acc * (1 - acc) / n)
+
+
+# ----------------------------------------------------------------------------- errors on the device
+
+def test_token_out_of_range_reported():
+    w = CASES[0][1]
+    d = synth.make(w)
+    d["last_token"] = d["last_token"].clone()
+    d["last_token"][2] = w.V + 5
+    p = sd.Params(B=w.B, K=w.K, V=w.V, r=w.r, dtype=w.dtype)
+    ws = sd.make_workspace(p)
+    dd = _dev(d)
+    o = sd.alloc_outputs(p)
+    sd.cycle(p, dd["base"], dd["target"], dd["U"], dd["W"], dd["last_token"], o["draft"], o["out"],
+             o["tau"], o["p_draft"], o["q_draft"], ws)
+    assert sd.sync_status(ws) == sd.SPEC_ERR_TOKEN_RANGE
+
+
+def test_wait_limit_gives_timeout_and_context_survives():
+    """A spin limit of one poll makes the first grid-barrier wait give up: the
+    kernel records SPEC_ERR_TIMEOUT and returns; the context stays usable."""
+    w = synth.Workload("to", B=8, K=3, V=32768, r=64, dtype="bf16", seed=66)
+    d = synth.make(w)
+    p = sd.Params(B=8, K=3, V=32768, r=64, dtype="bf16", spin_limit=1)
+    ws = sd.make_workspace(p)
+    dd = _dev(d)
+    o = sd.alloc_outputs(p)
+    sd.cycle(p, dd["base"], dd["target"], dd["U"], dd["W"], dd["last_token"], o["draft"], o["out"],
+             o["tau"], o["p_draft"], o["q_draft"], ws)
+    assert sd.sync_status(ws) == sd.SPEC_ERR_TIMEOUT
+    # same workspace after re-initialisation, normal limit: correct results
+    sd.workspace_init(ws)
+    g = gpu_cycle(w, d, dd=dd)
+    o2 = orc_cycle(w, d)
+    compare_cycle(g, o2, w.K)

@@ -18,6 +18,7 @@ SPEC_OK, SPEC_ERR_INVALID_ARG, SPEC_ERR_UNSUPPORTED, SPEC_ERR_CUDA = 0, -1, -2, 
 SPEC_ERR_TIMEOUT, SPEC_ERR_WORKSPACE, SPEC_ERR_TOKEN_RANGE = -4, -5, -6
 SPEC_F32, SPEC_BF16 = 0, 1
 SPEC_FLAG_FMA_BIAS = 1
+SPEC_FLAG_TRACE = 2
 
 # (name, restype, argtypes) of every exported symbol declared in include/*.h
 _P = ctypes.c_void_p
@@ -29,6 +30,7 @@ _SIGS = {
     "spec_verify_block": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_cycle": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_sync_status": (ctypes.c_int, [_P, _P]),
+    "spec_l2_persist": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
     "spec_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "spec_last_launch_count": (ctypes.c_int32, []),
     "spec_debug_philox": (ctypes.c_int, [_P, _P, _P, ctypes.c_int32, _P]),
@@ -162,6 +164,14 @@ def cycle(p: Params, base, target, U, W, last_token, draft, out, tau, p_draft, q
 
 def sync_status(ws, stream=None) -> int:
     return int(lib().spec_sync_status(_ptr(ws), _stream(stream)))
+
+
+def l2_persist(t, nbytes=None, stream=None):
+    """Keep tensor `t` (e.g. the Markov factor W) resident in L2 for kernels
+    launched on the stream; t=None clears the window."""
+    ptr = None if t is None else ctypes.c_void_p(t.data_ptr())
+    n = 0 if t is None else (t.numel() * t.element_size() if nbytes is None else nbytes)
+    _check(lib().spec_l2_persist(ptr, n, _stream(stream)), "spec_l2_persist")
 
 
 def last_launch_count() -> int:

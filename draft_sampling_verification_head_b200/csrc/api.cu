@@ -259,6 +259,7 @@ static spec_status run_cycle(const spec_params* p, int mode, const void* base, c
   L.seed = p->seed;
   L.cycle = p->cycle;
   L.spin = spin_of(p);
+  L.trace = (p->flags & SPEC_FLAG_TRACE) != 0;
   cudaError_t e = launch_cycle(L, g, header_of(ws), body_of(ws), g.tc ? &tmW : nullptr, &tmBase,
                                (cudaStream_t)stream);
   g_last_launches = 1;
@@ -321,6 +322,35 @@ spec_status spec_verify_block(const spec_params* p, const void* target, const vo
                       &launches);
   g_last_launches = launches;
   return e == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
+}
+
+spec_status spec_l2_persist(const void* ptr, size_t bytes, spec_stream_t stream) {
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaStreamAttrValue v;
+  memset(&v, 0, sizeof(v));
+  if (bytes == 0 || ptr == nullptr) {
+    v.accessPolicyWindow.num_bytes = 0;
+    if (cudaStreamSetAttribute(st, cudaStreamAttributeAccessPolicyWindow, &v) != cudaSuccess)
+      return SPEC_ERR_CUDA;
+    return cudaCtxResetPersistingL2Cache() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
+  }
+  int dev = 0, max_persist = 0, max_window = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&max_persist, cudaDevAttrMaxPersistingL2CacheSize, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&max_window, cudaDevAttrMaxAccessPolicyWindowSize, dev) != cudaSuccess)
+    return SPEC_ERR_CUDA;
+  if (max_persist <= 0 || max_window <= 0) return SPEC_ERR_UNSUPPORTED;
+  const size_t window = std::min(bytes, (size_t)max_window);
+  const size_t carve = std::min(window, (size_t)max_persist);
+  if (cudaDeviceSetLimit(cudaLimitPersistingL2CacheSize, carve) != cudaSuccess) return SPEC_ERR_CUDA;
+  v.accessPolicyWindow.base_ptr = const_cast<void*>(ptr);
+  v.accessPolicyWindow.num_bytes = window;
+  v.accessPolicyWindow.hitRatio = (float)carve / (float)window;
+  v.accessPolicyWindow.hitProp = cudaAccessPropertyPersisting;
+  v.accessPolicyWindow.missProp = cudaAccessPropertyStreaming;
+  return cudaStreamSetAttribute(st, cudaStreamAttributeAccessPolicyWindow, &v) == cudaSuccess
+             ? SPEC_OK
+             : SPEC_ERR_CUDA;
 }
 
 spec_status spec_debug_philox(const uint32_t* ctr, const uint32_t* key, uint32_t* out, int32_t n,

@@ -145,14 +145,16 @@ SPEC_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
                "r"(bytes)
                : "memory");
 }
+// One poll; the thread may be suspended in hardware for up to ~1 us while the
+// phase is incomplete, so waiting warps do not take issue slots.
 SPEC_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(1000u)
       : "memory");
   return ok != 0;
 }
@@ -174,6 +176,11 @@ SPEC_DEV bool mbar_drain(uint64_t* bar, uint32_t parity) {
   for (uint64_t it = 0; it < kDrainPolls; ++it)
     if (mbar_try_wait(bar, parity)) return true;
   return false;
+}
+
+// Bulk prefetch of [p, p + bytes) into L2 (16-byte aligned, size a multiple of 16).
+SPEC_DEV void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 SPEC_DEV void fence_proxy_async_smem() {
@@ -337,13 +344,14 @@ SPEC_DEV float warp_max(float v) {
 // s = sum exp2((x - m) * k) with k = log2(e) / T.  Differences x - m are taken
 // before scaling so that the dominant terms carry no rounding from the scale.
 // Combine two such pairs.
+// Branch-free: one exp2, of the smaller max relative to the larger.
 SPEC_DEV void ms_combine(float& m, float& s, float m2, float s2, float k) {
-  if (m2 > m) {
-    s = s2 + s * exp2f((m - m2) * k);
-    m = m2;
-  } else if (m2 > -INFINITY) {
-    s = s + s2 * exp2f((m2 - m) * k);
-  }
+  const bool first = m >= m2;
+  const float mb = first ? m : m2, ml = first ? m2 : m;
+  const float sb = first ? s : s2, sl = first ? s2 : s;
+  const float e = (ml == -INFINITY) ? 0.f : exp2f((ml - mb) * k);
+  m = mb;
+  s = fmaf(sl, e, sb);
 }
 
 // Arg-max pair with lowest-index tie-break.

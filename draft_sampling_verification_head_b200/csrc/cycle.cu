@@ -51,6 +51,8 @@ constexpr int kNS = 8;              // W ring stages
 constexpr int kNBS = 2;             // base tile ring stages
 constexpr int kMaxNC = 32;
 constexpr int kWStage = kCH * 64 * 2;  // 16 KB: 128 tokens x 64 rank, bf16
+constexpr int kMaxG = 160;          // CTAs a launch may use (>= SM count); partial-row stride
+constexpr int kOwnBatch = 8;        // owned rows scanned together by one warp
 constexpr unsigned FULL = 0xffffffffu;
 
 struct Args {
@@ -68,11 +70,12 @@ struct Args {
   float* q_draft;
   float* biased_out;
   WsHeader* hdr;
-  float2* dpart;     // [2][K+1][N][G]
-  float2* tpart;     // [2][K+1][N][G]
+  float2* dpart;     // [2][K+1][N][kMaxG]
+  float2* tpart;     // [2][K+1][N][kMaxG]
   int32_t* tokens;   // [2][K][N]
   int32_t* accf;     // [2][K][N]
   StopInfo* stopinfo;// [2][N]
+  uint64_t* trace;   // [K+2][kTracePhases] device timeline of CTA 0, or null
   int B, K, V, r, G, nc, nchunks, mode, greedy, ngroups;
   float k;           // log2(e) / T (1 in greedy mode)
   uint64_t seed, cycle, spin;
@@ -94,11 +97,49 @@ struct Ctl {
   int32_t tok[N];
   float M[N], S[N];     // global draft stats of the current step
   float zM[N], zS[N];   // draft stats of the stop row
-  float Mt[N], St[N];   // target stats for the final step
-  float Tg[N];          // owner target (prefix-relative) during the final step
+  float Mt[N], St[N];   // target stats (row i during a step, stop row / row K at the end)
+  int16_t wlist[8][N];  // owned rows per compute warp
+  int32_t wcount[8];
 };
 
 SPEC_DEV void named_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+SPEC_DEV uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Eight consecutive logits as raw 16-byte loads (streaming, L1 bypass).
+template <typename T>
+struct Raw8;
+template <>
+struct Raw8<__nv_bfloat16> {
+  uint4 a;
+};
+template <>
+struct Raw8<float> {
+  float4 a, b;
+};
+SPEC_DEV Raw8<__nv_bfloat16> raw_load(const __nv_bfloat16* p) {
+  return Raw8<__nv_bfloat16>{__ldcs(reinterpret_cast<const uint4*>(p))};
+}
+SPEC_DEV Raw8<float> raw_load(const float* p) {
+  return Raw8<float>{__ldcs(reinterpret_cast<const float4*>(p)),
+                     __ldcs(reinterpret_cast<const float4*>(p) + 1)};
+}
+SPEC_DEV void raw_expand(const Raw8<__nv_bfloat16>& r, float* x) {
+  const uint32_t w[4] = {r.a.x, r.a.y, r.a.z, r.a.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    x[2 * j] = __uint_as_float(w[j] << 16);
+    x[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+  }
+}
+SPEC_DEV void raw_expand(const Raw8<float>& r, float* x) {
+  x[0] = r.a.x; x[1] = r.a.y; x[2] = r.a.z; x[3] = r.a.w;
+  x[4] = r.b.x; x[5] = r.b.y; x[6] = r.b.z; x[7] = r.b.w;
+}
 
 template <typename T>
 SPEC_DEV float to_f(T x);
@@ -109,22 +150,6 @@ SPEC_DEV float to_f<float>(float x) {
 template <>
 SPEC_DEV float to_f<__nv_bfloat16>(__nv_bfloat16 x) {
   return __bfloat162float(x);
-}
-
-SPEC_DEV void load8(const __nv_bfloat16* p, float* x) {
-  const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    x[2 * j] = __uint_as_float(w[j] << 16);
-    x[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-  }
-}
-SPEC_DEV void load8(const float* p, float* x) {
-  const float4 a = __ldcs(reinterpret_cast<const float4*>(p));
-  const float4 b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
-  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
 }
 
 // ---- transposing butterflies: NCOL column values per lane -> lane L holds
@@ -377,6 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             break;
           }
           tc_fence_after();
+          if (a.trace && cta == 0 && g == 0) a.trace[(size_t)min(s, K) * kTracePhases + 9] = globaltimer_ns();
           for (int cl = 0; cl < ncc && ok; ++cl) {
             const uint32_t dcol = taddr + (uint32_t)(cl * N);
             for (int kb = 0; kb < nkb; ++kb) {
@@ -400,6 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             }
             if (ok) umma_commit(&ctl->dfull[cl]);
           }
+          if (a.trace && cta == 0 && g == 0) a.trace[(size_t)min(s, K) * kTracePhases + 10] = globaltimer_ns();
         }
       }
       umma_commit(&ctl->mmadone);
@@ -459,89 +486,206 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
     const float NaNf = __int_as_float(0x7fc00000);
     const int vslice_lo = chunk0 * kCH;
     const int vslice_hi = min(V, (chunk0 + ncc) * kCH);
+    // device timeline (trace flag): CTA 0, first group, one row of marks per step
+    uint64_t* trace = (a.trace != nullptr && cta == 0 && tid == 0) ? a.trace : nullptr;
+    auto mark = [&](int g, int step, int phase) {
+      if (trace && g == 0) trace[(size_t)step * kTracePhases + phase] = globaltimer_ns();
+    };
 
-    // Target row statistics over this CTA's slice for rows still alive.
+    // Target row statistics over this CTA's slice for the rows still alive.
+    // Each warp takes RB rows at a time and issues every 16-byte load of the
+    // batch before using any, so the loads overlap.
     auto target_row_stats = [&](int g, int par, int row, int nb_g) {
-      for (int n = warp; n < nb_g; n += 8) {
-        if (!ctl->alive[n]) continue;
-        const int b = g * N + n;
-        const T* t = target + ((int64_t)b * (K + 1) + row) * V;
-        float m = -INFINITY, s = 0.f, av = -INFINITY;
-        int32_t ai = 0x7fffffff;
-        for (int v = vslice_lo + lane * 8; v < vslice_hi; v += 256) {
-          float e[8];
-          load8(t + v, e);
-          float lm = e[0];
+      constexpr int RB = 2;
+      constexpr int VPL = 4;
+      for (int nb = warp; nb < nb_g; nb += 8 * RB) {
+        int rn[RB];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (e[j] > av) {
-              av = e[j];
-              ai = v + j;
-            }
-            lm = fmaxf(lm, e[j]);
-          }
-          if (!a.greedy) {
-            if (lm > m) {
-              s *= exp2f((m - lm) * k);
-              m = lm;
+        for (int r = 0; r < RB; ++r) {
+          const int n = nb + 8 * r;
+          rn[r] = (n < nb_g && ctl->alive[n]) ? n : -1;
+        }
+        float m[RB], s[RB], av[RB];
+        int32_t ai[RB];
+#pragma unroll
+        for (int r = 0; r < RB; ++r) {
+          m[r] = -INFINITY;
+          s[r] = 0.f;
+          av[r] = -INFINITY;
+          ai[r] = 0x7fffffff;
+        }
+        for (int vb = vslice_lo; vb < vslice_hi; vb += VPL * 256) {
+          Raw8<T> x[RB][VPL];
+#pragma unroll
+          for (int r = 0; r < RB; ++r)
+#pragma unroll
+            for (int u = 0; u < VPL; ++u) {
+              const int v = vb + u * 256 + lane * 8;
+              const int vv = v < vslice_hi ? v : vslice_lo;
+              const int nn = rn[r] >= 0 ? rn[r] : 0;
+              x[r][u] = raw_load(target + ((int64_t)(g * N + nn) * (K + 1) + row) * V + vv);
             }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) s += exp2f((e[j] - m) * k);
-          }
+          for (int r = 0; r < RB; ++r)
+#pragma unroll
+            for (int u = 0; u < VPL; ++u) {
+              const int v = vb + u * 256 + lane * 8;
+              if (rn[r] < 0 || v >= vslice_hi) continue;
+              float e[8];
+              raw_expand(x[r][u], e);
+              float lm = e[0];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                if (e[j] > av[r]) {
+                  av[r] = e[j];
+                  ai[r] = v + j;
+                }
+                lm = fmaxf(lm, e[j]);
+              }
+              if (!a.greedy) {
+                if (lm > m[r]) {
+                  s[r] *= exp2f((m[r] - lm) * k);
+                  m[r] = lm;
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) s[r] += exp2f((e[j] - m[r]) * k);
+              }
+            }
         }
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) {
-          const float m2 = __shfl_xor_sync(FULL, m, off), s2 = __shfl_xor_sync(FULL, s, off);
-          const float a2 = __shfl_xor_sync(FULL, av, off);
-          const int32_t i2 = __shfl_xor_sync(FULL, ai, off);
-          ms_combine(m, s, m2, s2, k);
-          amax_combine(av, ai, a2, i2);
-        }
-        if (lane == 0) {
-          float2* dst = a.tpart + (((int64_t)par * (K + 1) + row) * N + n) * G + cta;
-          *dst = a.greedy ? make_float2(av, __int_as_float(ai)) : make_float2(m, s);
+        for (int r = 0; r < RB; ++r) {
+          if (rn[r] < 0) continue;  // warp-uniform
+#pragma unroll
+          for (int off = 16; off >= 1; off >>= 1) {
+            const float m2 = __shfl_xor_sync(FULL, m[r], off), s2 = __shfl_xor_sync(FULL, s[r], off);
+            const float a2 = __shfl_xor_sync(FULL, av[r], off);
+            const int32_t i2 = __shfl_xor_sync(FULL, ai[r], off);
+            ms_combine(m[r], s[r], m2, s2, k);
+            amax_combine(av[r], ai[r], a2, i2);
+          }
+          if (lane == 0)
+            a.tpart[(((int64_t)par * (K + 1) + row) * N + rn[r]) * kMaxG + cta] =
+                a.greedy ? make_float2(av[r], __int_as_float(ai[r])) : make_float2(m[r], s[r]);
         }
       }
     };
 
-    // Combine the G target partials of one row for batch-row slot n (one warp).
-    auto warp_target_stats = [&](int par, int row, int n, float& M, float& S, int32_t& amax) {
-      float m = -INFINITY, s = 0.f, av = -INFINITY;
-      int32_t ai = 0x7fffffff;
-      for (int c = lane; c < G; c += 32) {
-        const float2 p = __ldcg(a.tpart + (((int64_t)par * (K + 1) + row) * N + n) * G + c);
-        if (a.greedy)
-          amax_combine(av, ai, p.x, __float_as_int(p.y));
-        else
-          ms_combine(m, s, p.x, p.y, k);
+    // ---- combine of the G per-CTA partials of one batch row: TPB threads per
+    // row, each holding a contiguous slice of the partials in registers (all
+    // loads in flight together).  Identical arithmetic in every CTA.
+    constexpr int MAXC = kMaxG / TPB;  // partials per thread (even: 16-byte loads)
+    static_assert(MAXC % 2 == 0, "partial slices are read as float4");
+    const int grp_n = tid / TPB, grp_sub = tid % TPB;
+    const int c_lo = grp_sub * MAXC;
+    const int c_hi = min(G, c_lo + MAXC);
+    // Unconditional 16-byte loads over the padded row (entries past G or of
+    // rows not in use are replaced afterwards), so all are in flight together.
+    auto load_slice = [&](const float2* pp, bool on, float2 (&reg)[MAXC], float2 dflt) {
+      const float4* p4 = reinterpret_cast<const float4*>(pp + c_lo);
+#pragma unroll
+      for (int j = 0; j < MAXC / 2; ++j) {
+        const float4 q = __ldcg(p4 + j);
+        reg[2 * j] = make_float2(q.x, q.y);
+        reg[2 * j + 1] = make_float2(q.z, q.w);
       }
 #pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) {
-        const float m2 = __shfl_xor_sync(FULL, m, off), s2 = __shfl_xor_sync(FULL, s, off);
+      for (int j = 0; j < MAXC; ++j)
+        if (!(on && c_lo + j < c_hi)) reg[j] = dflt;
+    };
+    // (m, s) partials -> global M, S (valid in every thread of the group)
+    auto group_ms = [&](const float2 (&reg)[MAXC], float& M, float& S) {
+      float m = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < MAXC; ++j) m = fmaxf(m, reg[j].x);
+#pragma unroll
+      for (int off = TPB / 2; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
+      float loc = 0.f;
+#pragma unroll
+      for (int j = 0; j < MAXC; ++j)
+        if (reg[j].y > 0.f) loc += reg[j].y * exp2f((reg[j].x - m) * k);
+      float sum = loc;
+#pragma unroll
+      for (int off = TPB / 2; off >= 1; off >>= 1) sum += __shfl_xor_sync(FULL, sum, off);
+      M = m;
+      S = sum;
+    };
+    auto group_amax = [&](const float2 (&reg)[MAXC], float& av, int32_t& ai) {
+      av = -INFINITY;
+      ai = 0x7fffffff;
+#pragma unroll
+      for (int j = 0; j < MAXC; ++j) amax_combine(av, ai, reg[j].x, __float_as_int(reg[j].y));
+#pragma unroll
+      for (int off = TPB / 2; off >= 1; off >>= 1) {
         const float a2 = __shfl_xor_sync(FULL, av, off);
         const int32_t i2 = __shfl_xor_sync(FULL, ai, off);
-        ms_combine(m, s, m2, s2, k);
         amax_combine(av, ai, a2, i2);
       }
-      M = m;
-      S = s;
-      amax = ai;
+    };
+    // Inverse-CDF owner among the G CTAs for weights w_c (given by wfun(j)),
+    // scanned in ascending c; returns true in the one thread whose slice holds
+    // the owner, with the owner index and the mass before it.
+    // weight of a partial: wmode 0 -> s * exp2((m - M) k) (softmax partials),
+    // 1 -> .x (residual mass), 2 -> .y (target mass)
+    auto pweight = [&](const float2& p, int wmode, float M) {
+      if (wmode == 0) return p.y > 0.f ? p.y * exp2f((p.x - M) * k) : 0.f;
+      return wmode == 1 ? p.x : p.y;
+    };
+    auto group_owner = [&](const float2 (&reg)[MAXC], int wmode, float M, float tgt, int& own,
+                           float& before, bool& fallback) {
+      float loc = 0.f;
+#pragma unroll
+      for (int j = 0; j < MAXC; ++j) loc += pweight(reg[j], wmode, M);
+      float incl = loc;
+#pragma unroll
+      for (int o = 1; o < TPB; o <<= 1) {
+        const float y = __shfl_up_sync(FULL, incl, o, TPB);
+        if (grp_sub >= o) incl += y;
+      }
+      float cum = incl - loc;
+      int found = 0x7fffffff, lastpos = -1;
+      before = 0.f;
+#pragma unroll
+      for (int j = 0; j < MAXC; ++j) {
+        if (c_lo + j >= c_hi) continue;
+        const float wj = pweight(reg[j], wmode, M);
+        if (wj > 0.f) lastpos = c_lo + j;
+        if (found == 0x7fffffff && cum + wj > tgt) {
+          found = c_lo + j;
+          before = cum;
+        }
+        cum += wj;
+      }
+      int o2 = found;
+#pragma unroll
+      for (int off = TPB / 2; off >= 1; off >>= 1) o2 = min(o2, __shfl_xor_sync(FULL, o2, off));
+      int lp = lastpos;
+#pragma unroll
+      for (int off = TPB / 2; off >= 1; off >>= 1) lp = max(lp, __shfl_xor_sync(FULL, lp, off));
+      fallback = o2 == 0x7fffffff;
+      own = fallback ? lp : o2;
+      return fallback ? (lastpos == own && own >= 0) : (found == own);
     };
 
     // Gather U[prev] rows (ctl->prev) into the B operand.
     auto gather_u = [&](int nb_g) {
       if (TC) {
         const int cpr = a.r / 8;  // 16-byte chunks per row
-        for (int idx = tid; idx < N * cpr; idx += kComputeThreads) {
+        constexpr int kIt = N * 32 / kComputeThreads;  // r <= 256: at most 32 chunks per row
+        uint4 val[kIt];
+#pragma unroll
+        for (int t = 0; t < kIt; ++t) {  // all loads first, from clamped (valid) rows
+          const int idx = tid + t * kComputeThreads;
+          const int n = min(idx / cpr, N - 1), c = idx % cpr;
+          val[t] = __ldg(reinterpret_cast<const uint4*>(Ug + (size_t)ctl->prev[n] * a.r) + c);
+        }
+#pragma unroll
+        for (int t = 0; t < kIt; ++t) {
+          const int idx = tid + t * kComputeThreads;
           const int n = idx / cpr, c = idx % cpr;
-          uint4 val = make_uint4(0, 0, 0, 0);
-          if (n < nb_g) {
-            const int p = ctl->prev[n];
-            val = __ldg(reinterpret_cast<const uint4*>(Ug + (size_t)p * a.r) + c);
-          }
+          if (idx >= N * cpr) continue;
           const int ka = c >> 3, j = c & 7;
           *reinterpret_cast<uint4*>(sU + (size_t)ka * N * 128 + n * 128 + ((j ^ (n & 7)) << 4)) =
-              val;
+              n < nb_g ? val[t] : make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
       } else {
@@ -592,6 +736,68 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
       return pos ? 31 - __clz(pos) : 0;
     };
 
+    // Bucket walk for every owned row (one thread each), then per-warp work
+    // lists: a row goes to one of the two warps of its bucket's quadrant.
+    // `mass(n, cl, q)` gives the bucket weight in the owner's scale.
+    // fin = false: softmax buckets (m, s) in the scale of ctl->M[n];
+    // fin = true: residual / target mass buckets, chosen by ctl->S[n] != 0.
+    auto bucket_mass = [&](int n, int cl, int q, bool fin) {
+      const float2 p = sBucket[((size_t)cl * 4 + q) * N + n];
+      if (!fin) return p.y > 0.f ? p.y * exp2f((p.x - ctl->M[n]) * k) : 0.f;
+      return ctl->S[n] != 0.f ? p.y : p.x;
+    };
+    auto walk_and_assign = [&](bool fin) {
+      const int n_owned = ctl->n_owned;
+      const int nbk = ncc * 4;  // buckets in ascending token order
+      for (int o = warp; o < n_owned; o += 8) {  // one warp per owned row
+        const int n = ctl->owned[o];
+        const float tin = ctl->obtarget[o];
+        float carry = 0.f;
+        int pick = -1, lastb = -1;
+        float tin_in = INFINITY;
+        for (int b0 = 0; b0 < nbk && pick < 0; b0 += 32) {  // 32 buckets per pass
+          const int bk = b0 + lane;
+          const float w = bk < nbk ? bucket_mass(n, bk >> 2, bk & 3, fin) : 0.f;
+          float incl = w;
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(FULL, incl, off);
+            if (lane >= off) incl += y;
+          }
+          const unsigned cross = __ballot_sync(FULL, carry + incl > tin);
+          const unsigned pos = __ballot_sync(FULL, w > 0.f);
+          if (pos) lastb = b0 + 31 - __clz(pos);
+          if (cross) {
+            const int l = __ffs(cross) - 1;
+            pick = b0 + l;
+            tin_in = tin - (carry + __shfl_sync(FULL, incl - w, l));
+          }
+          carry += __shfl_sync(FULL, incl, 31);
+        }
+        if (lane == 0) {
+          if (pick < 0) {
+            pick = lastb < 0 ? 0 : lastb;
+            tin_in = INFINITY;
+          }
+          ctl->obucket[o] = pick;
+          ctl->obtarget[o] = tin_in;
+        }
+      }
+      named_sync();
+      if (tid < 4) {
+        int c0 = 0, c1 = 0, alt = 0;
+        for (int o = 0; o < n_owned; ++o) {
+          if ((ctl->obucket[o] & 3) != tid) continue;
+          if (alt) ctl->wlist[tid + 4][c1++] = (int16_t)o;
+          else ctl->wlist[tid][c0++] = (int16_t)o;
+          alt ^= 1;
+        }
+        ctl->wcount[tid] = c0;
+        ctl->wcount[tid + 4] = c1;
+      }
+      named_sync();
+    };
+
     for (int g = 0; g < a.ngroups && !failed; ++g) {
       const int par = g & 1;
       const int nb_g = min(N, a.B - g * N);
@@ -611,10 +817,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           a.q_draft[(int64_t)(g * N) * K + idx] = NaNf;
       }
       named_sync();
+      mark(g, K + 1, 0);
       if (a.mode == MODE_CYCLE) target_row_stats(g, par, 0, nb_g);
+      mark(g, K + 1, 1);
 
       for (int i = 0; i < K; ++i) {
         // ---------------- gather the Markov rows for this step
+        mark(g, i, 0);
         for (int n = tid; n < N; n += kComputeThreads) {
           int p = 0;
           if (n < nb_g) {
@@ -628,11 +837,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
         }
         named_sync();
         gather_u(nb_g);
+        // pull the next target row of every live batch row into L2 now; the
+        // background pass reads it while this step's barrier completes
+        if (a.mode == MODE_CYCLE && tid < nb_g && ctl->alive[tid])
+          prefetch_l2_bulk(target + ((int64_t)(g * N + tid) * (K + 1) + i + 1) * V + vslice_lo,
+                           (uint32_t)((vslice_hi - vslice_lo) * sizeof(T)));
+        mark(g, i, 1);
 
         // ---------------- epilogue: z = base + bias, bucket statistics
+        uint64_t t_wait = 0;
         for (int cl = 0; cl < ncc; ++cl) {
           float d[NCOL];
+          const uint64_t t_w0 = trace ? globaltimer_ns() : 0;
           bias_tile(cl, d);
+          if (trace) t_wait += globaltimer_ns() - t_w0;
           const uint32_t bslot = Lb % kNBS;
           if (!mbar_wait_bounded(&ctl->bfull[bslot], (Lb / kNBS) & 1, a.spin, &hdr->abort))
             soft_fail(SPEC_ERR_TIMEOUT, SITE_MBAR_BASE, cta, i);
@@ -641,10 +859,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           const int v = (chunk0 + cl) * kCH + vl;
           const bool valid = v < V;
 #pragma unroll
-          for (int j = 0; j < NCOL; ++j) d[j] = valid ? d[j] + to_f<T>(bt[(n0 + j) * kCH + vl]) : -INFINITY;
+          for (int j = 0; j < NCOL; ++j)
+            d[j] = valid ? d[j] + to_f<T>(bt[(n0 + j) * kCH + vl]) : -INFINITY;
           __syncwarp();
           if (lane == 0) mbar_arrive(&ctl->bempty[bslot]);
           ++Lb;
+          // z replaces the bias in tensor memory: the owner scan reads it back
+          if (!a.greedy)
+            tmem_st_cols<NCOL>(taddr + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(cl * N + n0), d);
           if (a.biased_out && valid) {
 #pragma unroll
             for (int j = 0; j < NCOL; ++j) {
@@ -668,126 +890,121 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             if ((lane & (32 / NCOL - 1)) == 0) bk[n0 + lane / (32 / NCOL)] = make_float2(d[0], s[0]);
           }
         }
+        tc_fence_before();  // z stores above are read by other warps after the barrier
         named_sync();
-        // ---------------- CTA partial per batch row
-        for (int n = tid; n < N; n += kComputeThreads) {
+        tc_fence_after();
+        mark(g, i, 2);
+        if (trace && g == 0) trace[(size_t)i * kTracePhases + 11] = t_wait;
+        // ---------------- CTA partial per batch row (TPB threads per row)
+        {
+          const int n = grp_n;
           float m = -INFINITY, s = 0.f;
           int32_t ai = 0x7fffffff;
-          for (int cl = 0; cl < ncc; ++cl)
-            for (int q = 0; q < 4; ++q) {
-              const float2 p = sBucket[((size_t)cl * 4 + q) * N + n];
-              if (a.greedy)
-                amax_combine(m, ai, p.x, __float_as_int(p.y));
-              else
-                ms_combine(m, s, p.x, p.y, k);
-            }
-          a.dpart[(((int64_t)par * (K + 1) + i) * N + n) * G + cta] =
-              a.greedy ? make_float2(m, __int_as_float(ai)) : make_float2(m, s);
+          for (int bk = grp_sub; bk < ncc * 4; bk += TPB) {
+            const float2 p = sBucket[(size_t)bk * N + n];
+            if (a.greedy)
+              amax_combine(m, ai, p.x, __float_as_int(p.y));
+            else
+              ms_combine(m, s, p.x, p.y, k);
+          }
+#pragma unroll
+          for (int off = TPB / 2; off >= 1; off >>= 1) {
+            const float m2 = __shfl_xor_sync(FULL, m, off), s2 = __shfl_xor_sync(FULL, s, off);
+            const int32_t i2 = __shfl_xor_sync(FULL, ai, off);
+            if (a.greedy)
+              amax_combine(m, ai, m2, i2);
+            else
+              ms_combine(m, s, m2, s2, k);
+          }
+          if (grp_sub == 0)
+            a.dpart[(((int64_t)par * (K + 1) + i) * N + n) * kMaxG + cta] =
+                a.greedy ? make_float2(m, __int_as_float(ai)) : make_float2(m, s);
         }
         grid_arrive();
+        mark(g, i, 3);
         // background while the barrier completes: next target row, rows alive so far
         if (a.mode == MODE_CYCLE) target_row_stats(g, par, i + 1, nb_g);
+        mark(g, i, 4);
         if (!grid_wait()) {
           failed = true;
           break;
         }
+        mark(g, i, 5);
 
         // ---------------- combine partials: every CTA, same order
         if (tid == 0) ctl->n_owned = 0;
         named_sync();
         {
-          const int n = tid / TPB, sub = tid % TPB;
-          const int c_lo = (int)(((int64_t)G * sub) / TPB), c_hi = (int)(((int64_t)G * (sub + 1)) / TPB);
-          const float2* pp = a.dpart + (((int64_t)par * (K + 1) + i) * N + n) * G;
+          const int n = grp_n;
+          const bool row_on = n < nb_g;
+          float2 reg[MAXC];
+          load_slice(a.dpart + (((int64_t)par * (K + 1) + i) * N + n) * kMaxG, row_on, reg,
+                     a.greedy ? make_float2(-INFINITY, __int_as_float(0x7fffffff))
+                              : make_float2(-INFINITY, 0.f));
           if (a.greedy) {
-            float av = -INFINITY;
-            int32_t ai = 0x7fffffff;
-            for (int c = c_lo; c < c_hi; ++c) {
-              const float2 p = __ldcg(pp + c);
-              amax_combine(av, ai, p.x, __float_as_int(p.y));
-            }
-#pragma unroll
-            for (int off = TPB / 2; off >= 1; off >>= 1) {
-              const float a2 = __shfl_xor_sync(FULL, av, off);
-              const int32_t i2 = __shfl_xor_sync(FULL, ai, off);
-              amax_combine(av, ai, a2, i2);
-            }
-            if (sub == 0 && n < nb_g) ctl->tok[n] = ai;
-          } else {
-            float m = -INFINITY;
-            for (int c = c_lo; c < c_hi; ++c) m = fmaxf(m, __ldcg(pp + c).x);
-#pragma unroll
-            for (int off = TPB / 2; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
-            float loc = 0.f;
-            for (int c = c_lo; c < c_hi; ++c) {
-              const float2 p = __ldcg(pp + c);
-              loc += p.y * exp2f((p.x - m) * k);
-            }
-            float incl = loc;
-#pragma unroll
-            for (int o = 1; o < TPB; o <<= 1) {
-              const float y = __shfl_up_sync(FULL, incl, o, TPB);
-              if (sub >= o) incl += y;
-            }
-            const float S = __shfl_sync(FULL, incl, TPB - 1, TPB);
-            const int b = g * N + n;
-            const float u = philox_uniform(a.seed, a.cycle, (uint32_t)b, (uint32_t)i, TAG_DRAFT);
-            const float tgt = u * S;
-            float cum = incl - loc;
-            int found = 0x7fffffff, lastpos = -1;
-            float before = 0.f;
-            for (int c = c_lo; c < c_hi; ++c) {
-              const float2 p = __ldcg(pp + c);
-              const float w = p.y * exp2f((p.x - m) * k);
-              if (w > 0.f) lastpos = c;
-              if (found == 0x7fffffff && cum + w > tgt) {
-                found = c;
-                before = cum;
-              }
-              cum += w;
-            }
-            int own = found;
-#pragma unroll
-            for (int off = TPB / 2; off >= 1; off >>= 1) own = min(own, __shfl_xor_sync(FULL, own, off));
-            int lp = lastpos;
-#pragma unroll
-            for (int off = TPB / 2; off >= 1; off >>= 1) lp = max(lp, __shfl_xor_sync(FULL, lp, off));
-            const bool fallback = own == 0x7fffffff;
-            if (fallback) own = lp;
-            if (n < nb_g) {
-              if (sub == 0) {
-                ctl->M[n] = m;
-                ctl->S[n] = S;
-              }
-              if (own == cta && ((!fallback && found == own) || (fallback && lastpos == own))) {
-                const int slot = atomicAdd(&ctl->n_owned, 1);
-                ctl->owned[slot] = n;
-                ctl->obtarget[slot] = fallback ? INFINITY : tgt - before;
-              }
-            }
-          }
-        }
-        named_sync();
-
-        if (a.greedy) {
-          // arg-max drafts are known everywhere; verify against the target arg-max
-          if (a.mode == MODE_CYCLE) {
-            for (int n = warp; n < nb_g; n += 8) {
-              if (!ctl->alive[n]) continue;
-              float Mt, St;
-              int32_t am;
-              warp_target_stats(par, i, n, Mt, St, am);
-              if (lane == 0) {
+            float av;
+            int32_t ai;
+            group_amax(reg, av, ai);
+            if (grp_sub == 0 && row_on) ctl->tok[n] = ai;
+            if (a.mode == MODE_CYCLE) {
+              const bool al = row_on && ctl->alive[n];
+              load_slice(a.tpart + (((int64_t)par * (K + 1) + i) * N + n) * kMaxG, al, reg,
+                         make_float2(-INFINITY, __int_as_float(0x7fffffff)));
+              float tv;
+              int32_t tam;
+              group_amax(reg, tv, tam);
+              if (grp_sub == 0 && al) {
                 const int b = g * N + n;
-                const bool acc = am == ctl->tok[n];
-                if (cta == 0) a.out[(int64_t)b * (K + 1) + i] = acc ? ctl->tok[n] : am;
+                const bool acc = tam == ai;
+                if (cta == 0) a.out[(int64_t)b * (K + 1) + i] = acc ? ai : tam;
                 if (!acc) {
                   ctl->alive[n] = 0;
                   ctl->stoprow[n] = i;
                 }
               }
             }
+          } else {
+            float M, S;
+            group_ms(reg, M, S);
+            mark(g, i, 12);
+            const int b = g * N + n;
+            const float u = philox_uniform(a.seed, a.cycle, (uint32_t)b, (uint32_t)i, TAG_DRAFT);
+            const float tgt = u * S;
+            int own;
+            float before;
+            bool fb;
+            const bool holder = group_owner(reg, 0, M, tgt, own, before, fb);
+            mark(g, i, 13);
+            if (row_on) {
+              if (grp_sub == 0) {
+                ctl->M[n] = M;
+                ctl->S[n] = S;
+              }
+              if (holder && own == cta) {
+                const int slot = atomicAdd(&ctl->n_owned, 1);
+                ctl->owned[slot] = n;
+                ctl->obtarget[slot] = fb ? INFINITY : tgt - before;
+              }
+            }
+            if (a.mode == MODE_CYCLE) {
+              // target statistics of row i for the rows still alive (used by owners)
+              const bool al = row_on && ctl->alive[n];
+              load_slice(a.tpart + (((int64_t)par * (K + 1) + i) * N + n) * kMaxG, al, reg,
+                         make_float2(-INFINITY, 0.f));
+              float Mt, St;
+              group_ms(reg, Mt, St);
+              if (grp_sub == 0 && al) {
+                ctl->Mt[n] = Mt;
+                ctl->St[n] = St;
+              }
+              mark(g, i, 14);
+            }
           }
+        }
+        named_sync();
+        mark(g, i, 6);
+
+        if (a.greedy) {
           if (cta == 0)
             for (int n = tid; n < nb_g; n += kComputeThreads)
               if (a.draft) a.draft[(int64_t)(g * N + n) * K + i] = ctl->tok[n];
@@ -795,86 +1012,87 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           named_sync();
           if (TC && tid == 0) mbar_arrive(&ctl->tfree);
         } else {
-          // ---------------- owners: bucket walk, then one warp scans the bucket
-          const int n_owned = ctl->n_owned;
-          for (int o = tid; o < n_owned; o += kComputeThreads) {
-            const int n = ctl->owned[o];
-            const float M = ctl->M[n];
-            float tin = ctl->obtarget[o], acc = 0.f;
-            int pick = -1, lastb = 0;
-            for (int cl = 0; cl < ncc && pick < 0; ++cl)
-              for (int q = 0; q < 4; ++q) {
-                const float2 p = sBucket[((size_t)cl * 4 + q) * N + n];
-                const float w = p.y * exp2f((p.x - M) * k);
-                if (w > 0.f) lastb = cl * 4 + q;
-                if (acc + w > tin) {
-                  pick = cl * 4 + q;
-                  break;
-                }
-                acc += w;
-              }
-            if (pick < 0) {
-              pick = lastb;
-              tin = INFINITY;
-            } else {
-              tin -= acc;
+          // ---------------- owners: bucket walk, then batched bucket scans
+          walk_and_assign(false);
+          mark(g, i, 15);
+          const int cnt = ctl->wcount[warp];
+          for (int bs = 0; bs < cnt; bs += kOwnBatch) {
+            int oo[kOwnBatch];
+            float dv[kOwnBatch], td[kOwnBatch], zd[kOwnBatch], qd[kOwnBatch];
+            int dtok[kOwnBatch];
+#pragma unroll
+            for (int j = 0; j < kOwnBatch; ++j) {
+              oo[j] = bs + j < cnt ? ctl->wlist[warp][bs + j] : -1;
+              dtok[j] = 0;
             }
-            ctl->obucket[o] = pick;
-            ctl->obtarget[o] = tin;
-          }
-          named_sync();
-          int mine = 0;
-          for (int o = 0; o < n_owned; ++o) {
-            const int pick = ctl->obucket[o];
-            const int q = pick & 3, cl = pick >> 2;
-            if (q != q4) continue;
-            if (((mine++) & 1) != (warp >> 2)) continue;  // two warps per quadrant
-            const int n = ctl->owned[o];
-            const int b = g * N + n;
-            const float M = ctl->M[n], S = ctl->S[n];
-            float dv;
-            tmem_ld1(taddr + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(cl * N + n), &dv);
+#pragma unroll
+            for (int j = 0; j < kOwnBatch; ++j) {
+              dv[j] = 0.f;
+              if (oo[j] < 0) continue;
+              const int cl = ctl->obucket[oo[j]] >> 2, n = ctl->owned[oo[j]];
+              tmem_ld1(taddr + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(cl * N + n), &dv[j]);
+            }
             tmem_ld_wait();
-            const int v = (chunk0 + cl) * kCH + q4 * 32 + lane;
-            const bool valid = v < V;
-            const float z = valid ? dv + ld_elem(base, ((int64_t)b * K + i) * V + v) : -INFINITY;
-            const float e = valid ? exp2f((z - M) * k) : 0.f;
-            const int wl = bucket_scan(e, ctl->obtarget[o]);
-            const int dtok = (chunk0 + cl) * kCH + q4 * 32 + wl;
-            const float zd = __shfl_sync(FULL, z, wl);
-            const float qd = exp2f((zd - M) * k) / S;
-            int accept = 1;
-            float pd = NaNf, Mt = 0.f, St = 1.f;
-            const bool alive = a.mode == MODE_CYCLE && ctl->alive[n];
-            if (alive) {
-              int32_t am;
-              warp_target_stats(par, i, n, Mt, St, am);
-              const float td = ld_elem(target, ((int64_t)b * (K + 1) + i) * V + dtok);
-              pd = exp2f((td - Mt) * k) / St;
-              const float ratio = exp2f(((td - Mt) - (zd - M)) * k) * (S / St);
-              const float uacc = philox_uniform(a.seed, a.cycle, (uint32_t)b, (uint32_t)i, TAG_ACCEPT);
-              accept = uacc < fminf(ratio, 1.0f) ? 1 : 0;
+#pragma unroll
+            for (int j = 0; j < kOwnBatch; ++j) {
+              if (oo[j] < 0) continue;
+              const int cl = ctl->obucket[oo[j]] >> 2, n = ctl->owned[oo[j]];
+              const float M = ctl->M[n], S = ctl->S[n];
+              const int v = (chunk0 + cl) * kCH + q4 * 32 + lane;
+              const bool valid = v < V;
+              const float z = valid ? dv[j] : -INFINITY;  // z = base + bias, kept in tensor memory
+              const float e = valid ? exp2f((z - M) * k) : 0.f;
+              const int wl = bucket_scan(e, ctl->obtarget[oo[j]]);
+              dtok[j] = (chunk0 + cl) * kCH + q4 * 32 + wl;
+              zd[j] = __shfl_sync(FULL, z, wl);
+              qd[j] = exp2f((zd[j] - M) * k) / S;
             }
-            if (lane == 0) {
-              a.tokens[((int64_t)par * K + i) * N + n] = dtok;
-              a.accf[((int64_t)par * K + i) * N + n] = accept;
-              if (a.draft) a.draft[(int64_t)b * K + i] = dtok;
-              if (a.q_draft) a.q_draft[(int64_t)b * K + i] = qd;
+            const bool cyc = a.mode == MODE_CYCLE;
+#pragma unroll
+            for (int j = 0; j < kOwnBatch; ++j) {
+              const int oj = oo[j] < 0 ? 0 : oo[j];
+              const int n = min(ctl->owned[oj], nb_g - 1);
+              const int dt = oo[j] < 0 ? 0 : min(max(dtok[j], 0), V - 1);
+              td[j] = cyc ? ld_elem(target, ((int64_t)(g * N + n) * (K + 1) + i) * V + dt) : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < kOwnBatch; ++j) {
+              if (oo[j] < 0) continue;
+              const int n = ctl->owned[oo[j]];
+              const int b = g * N + n;
+              const float M = ctl->M[n], S = ctl->S[n];
+              const bool alive = cyc && ctl->alive[n];
+              int accept = 1;
+              float pd = NaNf;
               if (alive) {
-                if (a.p_draft) a.p_draft[(int64_t)b * K + i] = pd;
-                if (accept)
-                  a.out[(int64_t)b * (K + 1) + i] = dtok;
-                else
-                  a.stopinfo[(int64_t)par * N + n] = StopInfo{i, Mt, St, M, S};
+                const float Mt = ctl->Mt[n], St = ctl->St[n];
+                pd = exp2f((td[j] - Mt) * k) / St;
+                const float ratio = exp2f(((td[j] - Mt) - (zd[j] - M)) * k) * (S / St);
+                const float uacc = philox_uniform(a.seed, a.cycle, (uint32_t)b, (uint32_t)i, TAG_ACCEPT);
+                accept = uacc < fminf(ratio, 1.0f) ? 1 : 0;
               }
-              __threadfence();
+              if (lane == 0) {
+                a.tokens[((int64_t)par * K + i) * N + n] = dtok[j];
+                a.accf[((int64_t)par * K + i) * N + n] = accept;
+                if (a.draft) a.draft[(int64_t)b * K + i] = dtok[j];
+                if (a.q_draft) a.q_draft[(int64_t)b * K + i] = qd[j];
+                if (alive) {
+                  if (a.p_draft) a.p_draft[(int64_t)b * K + i] = pd;
+                  if (accept)
+                    a.out[(int64_t)b * (K + 1) + i] = dtok[j];
+                  else
+                    a.stopinfo[(int64_t)par * N + n] = StopInfo{i, ctl->Mt[n], ctl->St[n], M, S};
+                }
+              }
             }
           }
+          mark(g, i, 7);
           tc_fence_before();
           named_sync();
           if (TC && tid == 0) mbar_arrive(&ctl->tfree);
           if (tid == 0) {
             __threadfence();
+            const int n_owned = ctl->n_owned;
             if (n_owned) red_release_add_u32(&hdr->tok, (uint32_t)n_owned);
             tok_expected += (uint32_t)nb_g;
             if (!grid_wait_count(hdr, &hdr->tok, tok_expected, a.spin, SITE_TOKEN_WAIT) ||
@@ -883,6 +1101,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             __threadfence();
           }
           named_sync();
+          mark(g, i, 8);
           if (ctl->abort_local) {
             failed = true;
             break;
@@ -891,10 +1110,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             ctl->tok[n] = __ldcg(a.tokens + ((int64_t)par * K + i) * N + n);
             if (a.mode == MODE_CYCLE && ctl->alive[n] &&
                 !__ldcg(a.accf + ((int64_t)par * K + i) * N + n)) {
+              const uint32_t sl = (uint32_t)((vslice_hi - vslice_lo) * sizeof(T));
+              prefetch_l2_bulk(target + ((int64_t)(g * N + n) * (K + 1) + i) * V + vslice_lo, sl);
+              prefetch_l2_bulk(base + ((int64_t)(g * N + n) * K + i) * V + vslice_lo, sl);
               ctl->alive[n] = 0;
               ctl->stoprow[n] = i;
               ctl->zM[n] = ctl->M[n];
               ctl->zS[n] = ctl->S[n];
+              ctl->Mt[n] = __ldcg(&a.stopinfo[(int64_t)par * N + n].mt);
+              ctl->St[n] = __ldcg(&a.stopinfo[(int64_t)par * N + n].st);
             }
           }
           named_sync();
@@ -909,34 +1133,37 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
 
       if (a.mode == MODE_CYCLE) {
         // row-K target partials (written after the last barrier) become visible
+        mark(g, K, 0);
         if (!grid_barrier()) {
           failed = true;
           break;
         }
-        if (a.greedy) {
-          for (int n = warp; n < nb_g; n += 8) {
-            if (!ctl->alive[n]) continue;
+        mark(g, K, 1);
+        {
+          // target statistics of row K for the rows that accepted every draft
+          const int n = grp_n;
+          const bool al = n < nb_g && ctl->alive[n];
+          float2 reg[MAXC];
+          load_slice(a.tpart + (((int64_t)par * (K + 1) + K) * N + n) * kMaxG, al, reg,
+                     a.greedy ? make_float2(-INFINITY, __int_as_float(0x7fffffff))
+                              : make_float2(-INFINITY, 0.f));
+          if (a.greedy) {
+            float tv;
+            int32_t tam;
+            group_amax(reg, tv, tam);
+            if (grp_sub == 0 && al && cta == 0) a.out[(int64_t)(g * N + n) * (K + 1) + K] = tam;
+          } else {
             float Mt, St;
-            int32_t am;
-            warp_target_stats(par, K, n, Mt, St, am);
-            if (lane == 0 && cta == 0) a.out[(int64_t)(g * N + n) * (K + 1) + K] = am;
-          }
-        } else {
-          // ---------------- final step: residual at the stop row, or the bonus
-          for (int n = warp; n < nb_g; n += 8) {
-            if (ctl->alive[n]) {
-              float Mt, St;
-              int32_t am;
-              warp_target_stats(par, K, n, Mt, St, am);
-              if (lane == 0) {
-                ctl->Mt[n] = Mt;
-                ctl->St[n] = St;
-              }
-            } else if (lane == 0) {
-              ctl->Mt[n] = __ldcg(&a.stopinfo[(int64_t)par * N + n].mt);
-              ctl->St[n] = __ldcg(&a.stopinfo[(int64_t)par * N + n].st);
+            group_ms(reg, Mt, St);
+            if (grp_sub == 0 && al) {
+              ctl->Mt[n] = Mt;
+              ctl->St[n] = St;
             }
           }
+        }
+        named_sync();
+        if (!a.greedy) {
+          // ---------------- final step: residual at the stop row, or the bonus
           for (int n = tid; n < N; n += kComputeThreads) {
             int p = 0;
             if (n < nb_g && !ctl->alive[n]) {
@@ -949,166 +1176,148 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           }
           named_sync();
           gather_u(nb_g);
+          mark(g, K, 2);
           for (int cl = 0; cl < ncc; ++cl) {
             float d[NCOL];
             bias_tile(cl, d);
             const int v = (chunk0 + cl) * kCH + q4 * 32 + lane;
             const bool valid = v < V;
-            float R[NCOL], P[NCOL];
+            float tv[NCOL], bvv[NCOL];
+#pragma unroll
+            for (int j = 0; j < NCOL; ++j) {  // loads from clamped valid addresses
+              const int n = min(n0 + j, nb_g - 1);
+              const int b = g * N + n;
+              const int row = ctl->alive[n] ? K : ctl->stoprow[n];
+              const int vv = valid ? v : V - 1;
+              tv[j] = ld_elem(target, ((int64_t)b * (K + 1) + row) * V + vv);
+              bvv[j] = ld_elem(base, ((int64_t)b * K + min(row, K - 1)) * V + vv);
+            }
+            // residual mass r (into tv) and target mass p (into bvv), in place
 #pragma unroll
             for (int j = 0; j < NCOL; ++j) {
               const int n = n0 + j;
-              R[j] = 0.f;
-              P[j] = 0.f;
+              float r = 0.f, p = 0.f;
               if (valid && n < nb_g) {
-                const int b = g * N + n;
-                const int row = ctl->alive[n] ? K : ctl->stoprow[n];
-                const float t = ld_elem(target, ((int64_t)b * (K + 1) + row) * V + v);
-                const float p = exp2f((t - ctl->Mt[n]) * k) / ctl->St[n];
-                float r = p;
-                if (!ctl->alive[n]) {
-                  const float z = d[j] + ld_elem(base, ((int64_t)b * K + row) * V + v);
-                  r = fmaxf(p - exp2f((z - ctl->zM[n]) * k) / ctl->zS[n], 0.f);
-                }
-                R[j] = r;
-                P[j] = p;
+                p = exp2f((tv[j] - ctl->Mt[n]) * k) / ctl->St[n];
+                r = p;
+                if (!ctl->alive[n])
+                  r = fmaxf(p - exp2f((d[j] + bvv[j] - ctl->zM[n]) * k) / ctl->zS[n], 0.f);
               }
+              tv[j] = r;
+              bvv[j] = p;
             }
-            bfly_sum2<NCOL>(R, P, lane);
+            bfly_sum2<NCOL>(tv, bvv, lane);
             float2* bk = sBucket + ((size_t)cl * 4 + q4) * N;
-            if ((lane & (32 / NCOL - 1)) == 0) bk[n0 + lane / (32 / NCOL)] = make_float2(R[0], P[0]);
+            if ((lane & (32 / NCOL - 1)) == 0) bk[n0 + lane / (32 / NCOL)] = make_float2(tv[0], bvv[0]);
           }
           named_sync();
-          for (int n = tid; n < N; n += kComputeThreads) {
+          {
+            const int n = grp_n;
             float R = 0.f, P = 0.f;
-            for (int cl = 0; cl < ncc; ++cl)
-              for (int q = 0; q < 4; ++q) {
-                const float2 p = sBucket[((size_t)cl * 4 + q) * N + n];
-                R += p.x;
-                P += p.y;
-              }
-            a.dpart[(((int64_t)par * (K + 1) + K) * N + n) * G + cta] = make_float2(R, P);
+            for (int bk = grp_sub; bk < ncc * 4; bk += TPB) {
+              const float2 p = sBucket[(size_t)bk * N + n];
+              R += p.x;
+              P += p.y;
+            }
+#pragma unroll
+            for (int off = TPB / 2; off >= 1; off >>= 1) {
+              R += __shfl_xor_sync(FULL, R, off);
+              P += __shfl_xor_sync(FULL, P, off);
+            }
+            if (grp_sub == 0)
+              a.dpart[(((int64_t)par * (K + 1) + K) * N + n) * kMaxG + cta] = make_float2(R, P);
           }
+          mark(g, K, 3);
           if (!grid_barrier()) {
             failed = true;
             break;
           }
+          mark(g, K, 4);
           if (tid == 0) ctl->n_owned = 0;
           named_sync();
           {
-            const int n = tid / TPB, sub = tid % TPB;
-            const int c_lo = (int)(((int64_t)G * sub) / TPB), c_hi = (int)(((int64_t)G * (sub + 1)) / TPB);
-            const float2* pp = a.dpart + (((int64_t)par * (K + 1) + K) * N + n) * G;
-            float lr = 0.f, lpp = 0.f;
-            for (int c = c_lo; c < c_hi; ++c) {
-              const float2 p = __ldcg(pp + c);
-              lr += p.x;
-              lpp += p.y;
-            }
-            float ir = lr, ip = lpp;
+            const int n = grp_n;
+            const bool row_on = n < nb_g;
+            float2 reg[MAXC];
+            load_slice(a.dpart + (((int64_t)par * (K + 1) + K) * N + n) * kMaxG, row_on, reg,
+                       make_float2(0.f, 0.f));
+            float lr = 0.f, lp = 0.f;
 #pragma unroll
-            for (int o = 1; o < TPB; o <<= 1) {
-              const float yr = __shfl_up_sync(FULL, ir, o, TPB);
-              const float yp = __shfl_up_sync(FULL, ip, o, TPB);
-              if (sub >= o) {
-                ir += yr;
-                ip += yp;
-              }
+            for (int j = 0; j < MAXC; ++j) {
+              lr += reg[j].x;
+              lp += reg[j].y;
             }
-            const float Rt = __shfl_sync(FULL, ir, TPB - 1, TPB);
-            const float Pt = __shfl_sync(FULL, ip, TPB - 1, TPB);
+            float Rt = lr, Pt = lp;
+#pragma unroll
+            for (int off = TPB / 2; off >= 1; off >>= 1) {
+              Rt += __shfl_xor_sync(FULL, Rt, off);
+              Pt += __shfl_xor_sync(FULL, Pt, off);
+            }
             const bool use_p = !(Rt > 0.f);
-            const float tot = use_p ? Pt : Rt;
             const int b = g * N + n;
-            const int row = (n < nb_g && ctl->alive[n]) ? K : (n < nb_g ? ctl->stoprow[n] : 0);
+            const int row = (row_on && ctl->alive[n]) ? K : (row_on ? ctl->stoprow[n] : 0);
             const float u = philox_uniform(a.seed, a.cycle, (uint32_t)b, (uint32_t)row, TAG_RESAMPLE);
-            const float tgt = u * tot;
-            float cum = use_p ? ip - lpp : ir - lr;
-            int found = 0x7fffffff, lastpos = -1;
-            float before = 0.f;
-            for (int c = c_lo; c < c_hi; ++c) {
-              const float2 p = __ldcg(pp + c);
-              const float w = use_p ? p.y : p.x;
-              if (w > 0.f) lastpos = c;
-              if (found == 0x7fffffff && cum + w > tgt) {
-                found = c;
-                before = cum;
-              }
-              cum += w;
-            }
-            int own = found;
-#pragma unroll
-            for (int off = TPB / 2; off >= 1; off >>= 1) own = min(own, __shfl_xor_sync(FULL, own, off));
-            int lp = lastpos;
-#pragma unroll
-            for (int off = TPB / 2; off >= 1; off >>= 1) lp = max(lp, __shfl_xor_sync(FULL, lp, off));
-            const bool fallback = own == 0x7fffffff;
-            if (fallback) own = lp;
-            if (n < nb_g) {
-              if (sub == 0) ctl->S[n] = use_p ? 1.f : 0.f;  // which mass the scan uses
-              if (own == cta && ((!fallback && found == own) || (fallback && lastpos == own))) {
+            const float tgt = u * (use_p ? Pt : Rt);
+            int own;
+            float before;
+            bool fb;
+            const bool holder = group_owner(reg, use_p ? 2 : 1, 0.f, tgt, own, before, fb);
+            if (row_on) {
+              if (grp_sub == 0) ctl->S[n] = use_p ? 1.f : 0.f;  // which mass the scan uses
+              if (holder && own == cta) {
                 const int slot = atomicAdd(&ctl->n_owned, 1);
                 ctl->owned[slot] = n;
-                ctl->obtarget[slot] = fallback ? INFINITY : tgt - before;
+                ctl->obtarget[slot] = fb ? INFINITY : tgt - before;
               }
             }
           }
           named_sync();
-          const int n_owned = ctl->n_owned;
-          for (int o = tid; o < n_owned; o += kComputeThreads) {
-            const int n = ctl->owned[o];
-            const bool use_p = ctl->S[n] != 0.f;
-            float tin = ctl->obtarget[o], acc = 0.f;
-            int pick = -1, lastb = 0;
-            for (int cl = 0; cl < ncc && pick < 0; ++cl)
-              for (int q = 0; q < 4; ++q) {
-                const float2 p = sBucket[((size_t)cl * 4 + q) * N + n];
-                const float w = use_p ? p.y : p.x;
-                if (w > 0.f) lastb = cl * 4 + q;
-                if (acc + w > tin) {
-                  pick = cl * 4 + q;
-                  break;
-                }
-                acc += w;
-              }
-            if (pick < 0) {
-              pick = lastb;
-              tin = INFINITY;
-            } else {
-              tin -= acc;
+          walk_and_assign(true);
+          const int cnt = ctl->wcount[warp];
+          for (int bs = 0; bs < cnt; bs += kOwnBatch) {
+            int oo[kOwnBatch];
+            float dv[kOwnBatch], tvv[kOwnBatch], bvv[kOwnBatch];
+#pragma unroll
+            for (int j = 0; j < kOwnBatch; ++j) oo[j] = bs + j < cnt ? ctl->wlist[warp][bs + j] : -1;
+#pragma unroll
+            for (int j = 0; j < kOwnBatch; ++j) {
+              dv[j] = 0.f;
+              if (oo[j] < 0) continue;
+              const int cl = ctl->obucket[oo[j]] >> 2, n = ctl->owned[oo[j]];
+              tmem_ld1(taddr + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(cl * N + n), &dv[j]);
             }
-            ctl->obucket[o] = pick;
-            ctl->obtarget[o] = tin;
-          }
-          named_sync();
-          int mine = 0;
-          for (int o = 0; o < n_owned; ++o) {
-            const int pick = ctl->obucket[o];
-            const int q = pick & 3, cl = pick >> 2;
-            if (q != q4) continue;
-            if (((mine++) & 1) != (warp >> 2)) continue;
-            const int n = ctl->owned[o];
-            const int b = g * N + n;
-            const bool use_p = ctl->S[n] != 0.f;
-            const bool bonus = ctl->alive[n] != 0;
-            const int row = bonus ? K : ctl->stoprow[n];
-            float dv;
-            tmem_ld1(taddr + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(cl * N + n), &dv);
             tmem_ld_wait();
-            const int v = (chunk0 + cl) * kCH + q4 * 32 + lane;
-            float w = 0.f;
-            if (v < V) {
-              const float t = ld_elem(target, ((int64_t)b * (K + 1) + row) * V + v);
-              const float p = exp2f((t - ctl->Mt[n]) * k) / ctl->St[n];
-              w = p;
-              if (!bonus && !use_p) {
-                const float z = dv + ld_elem(base, ((int64_t)b * K + row) * V + v);
-                w = fmaxf(p - exp2f((z - ctl->zM[n]) * k) / ctl->zS[n], 0.f);
-              }
+#pragma unroll
+            for (int j = 0; j < kOwnBatch; ++j) {  // loads from clamped valid addresses
+              const int oj = oo[j] < 0 ? 0 : oo[j];
+              const int cl = ctl->obucket[oj] >> 2, n = min(ctl->owned[oj], nb_g - 1);
+              const int b = g * N + n;
+              const int row = ctl->alive[n] ? K : ctl->stoprow[n];
+              const int v = min((chunk0 + cl) * kCH + q4 * 32 + lane, V - 1);
+              tvv[j] = ld_elem(target, ((int64_t)b * (K + 1) + row) * V + v);
+              bvv[j] = ld_elem(base, ((int64_t)b * K + min(row, K - 1)) * V + v);
             }
-            const int wl = bucket_scan(w, ctl->obtarget[o]);
-            if (lane == 0) a.out[(int64_t)b * (K + 1) + row] = (chunk0 + cl) * kCH + q4 * 32 + wl;
+#pragma unroll
+            for (int j = 0; j < kOwnBatch; ++j) {
+              if (oo[j] < 0) continue;
+              const int cl = ctl->obucket[oo[j]] >> 2, n = ctl->owned[oo[j]];
+              const int b = g * N + n;
+              const bool use_p = ctl->S[n] != 0.f;
+              const bool bonus = ctl->alive[n] != 0;
+              const int row = bonus ? K : ctl->stoprow[n];
+              const int v = (chunk0 + cl) * kCH + q4 * 32 + lane;
+              float w = 0.f;
+              if (v < V) {
+                const float p = exp2f((tvv[j] - ctl->Mt[n]) * k) / ctl->St[n];
+                w = p;
+                if (!bonus && !use_p)
+                  w = fmaxf(p - exp2f((dv[j] + bvv[j] - ctl->zM[n]) * k) / ctl->zS[n], 0.f);
+              }
+              const int wl = bucket_scan(w, ctl->obtarget[oo[j]]);
+              if (lane == 0) a.out[(int64_t)b * (K + 1) + row] = (chunk0 + cl) * kCH + q4 * 32 + wl;
+            }
           }
+          mark(g, K, 5);
           tc_fence_before();
           named_sync();
           if (TC && tid == 0) mbar_arrive(&ctl->tfree);
@@ -1124,6 +1333,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           }
         }
         named_sync();
+        mark(g, K, 6);
       }
     }  // groups
     (void)soft_fail;
@@ -1210,6 +1420,10 @@ bool cycle_geometry(int B, int K, int V, int r, int dtype, uint32_t flags, int n
   g->nchunks = nchunks;
   g->nc = nc;
   g->G = (nchunks + nc - 1) / nc;
+  if (g->G > kMaxG) {
+    *why = "more CTAs than the kernel's partial buffers allow";
+    return false;
+  }
   g->N = N;
   g->tc = tc;
   g->smem = dtype == SPEC_BF16 ? (tc ? smem_for<__nv_bfloat16, true>(N, r, nc)
@@ -1227,11 +1441,13 @@ namespace {
 size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 }  // namespace
 
-// Workspace body: dpart | tpart | tokens | accf | stopinfo, each 256-byte aligned.
+// Workspace body: trace | dpart | tpart | tokens | accf | stopinfo, each 256-byte aligned.
+size_t cycle_trace_bytes(int K) { return a256(sizeof(uint64_t) * (size_t)(K + 2) * kTracePhases); }
 size_t cycle_ws_bytes(int K, const CycleGeom& g) {
-  const size_t part = sizeof(float2) * 2 * (size_t)(K + 1) * g.N * g.G;
+  const size_t part = sizeof(float2) * 2 * (size_t)(K + 1) * g.N * kMaxG;
   const size_t tok = sizeof(int32_t) * 2 * (size_t)K * g.N;
-  return 2 * a256(part) + 2 * a256(tok) + a256(sizeof(StopInfo) * 2 * g.N);
+  return cycle_trace_bytes(K) + 2 * a256(part) + 2 * a256(tok) +
+         a256(sizeof(StopInfo) * 2 * g.N);
 }
 
 cudaError_t launch_cycle(const CycleLaunch& L, const CycleGeom& g, WsHeader* hdr, uint8_t* body,
@@ -1252,8 +1468,10 @@ cudaError_t launch_cycle(const CycleLaunch& L, const CycleGeom& g, WsHeader* hdr
   a.q_draft = L.q_draft;
   a.biased_out = L.biased_out;
   a.hdr = hdr;
-  const size_t part = a256(sizeof(float2) * 2 * (size_t)(L.K + 1) * g.N * g.G);
+  const size_t part = a256(sizeof(float2) * 2 * (size_t)(L.K + 1) * g.N * kMaxG);
   const size_t tok = a256(sizeof(int32_t) * 2 * (size_t)L.K * g.N);
+  a.trace = L.trace ? reinterpret_cast<uint64_t*>(body) : nullptr;
+  body += cycle_trace_bytes(L.K);
   a.dpart = reinterpret_cast<float2*>(body);
   a.tpart = reinterpret_cast<float2*>(body + part);
   a.tokens = reinterpret_cast<int32_t*>(body + 2 * part);

@@ -55,6 +55,8 @@ struct CycleGeom {
 bool cycle_geometry(int B, int K, int V, int r, int dtype, uint32_t flags, int num_sms,
                     CycleGeom* g, const char** why);
 size_t cycle_ws_bytes(int K, const CycleGeom& g);
+constexpr int kTracePhases = 16;  // timeline slots per step
+size_t cycle_trace_bytes(int K);
 
 struct CycleLaunch {
   const void* base;
@@ -71,6 +73,7 @@ struct CycleLaunch {
   int B, K, V, r, dtype, mode, greedy;
   float temperature;
   uint64_t seed, cycle, spin;
+  bool trace;
 };
 
 cudaError_t launch_cycle(const CycleLaunch& L, const CycleGeom& g, WsHeader* hdr, uint8_t* body,

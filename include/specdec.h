@@ -78,6 +78,13 @@ typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 
 /* Flags */
 #define SPEC_FLAG_FMA_BIAS 1u  /* compute the Markov bias with fp32 FMAs instead of tensor cores */
+#define SPEC_FLAG_TRACE 2u     /* spec_cycle / spec_markov_bias_sample: record a device timeline.
+                                  CTA 0 writes %globaltimer (ns) into the workspace at byte offset
+                                  256 as uint64 [K+2][16]: row i < K = draft step i (slots: 0 start,
+                                  1 rows gathered, 2 epilogue done, 3 partials published, 4 target
+                                  rows streamed, 5 barrier passed, 6 partials combined, 7 owner
+                                  draws done, 8 tokens known), row K = final step, row K+1 =
+                                  prologue.  Only the first batch group is recorded. */
 
 typedef struct {
   int32_t B;             /* batch rows, >= 1 */
@@ -133,6 +140,14 @@ spec_status spec_cycle(const spec_params *p, const void *base, const void *targe
                        const void *W, const int32_t *last_token, int32_t *draft, int32_t *out,
                        int32_t *tau, float *p_draft, float *q_draft, void *workspace,
                        spec_stream_t stream);
+
+/* Keep [ptr, ptr + bytes) resident in L2 for kernels later launched on
+ * `stream` (a persisting access-policy window on the stream; the persisting
+ * L2 carve-out of the calling process's context is raised to fit, up to the
+ * device maximum).  Meant for the Markov factor W, which every draft step
+ * re-reads.  bytes = 0 removes the window and releases persisting lines.  The
+ * carve-out belongs to this process's context and ends with it. */
+spec_status spec_l2_persist(const void *ptr, size_t bytes, spec_stream_t stream);
 
 /* Synchronise `stream` and return the device-side status recorded in the
  * workspace by the calls issued on it (SPEC_OK if none failed). */

@@ -30,6 +30,7 @@ _SIGS = {
     "spec_verify_block": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_cycle": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_sync_status": (ctypes.c_int, [_P, _P]),
+    "spec_cycle_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_l2_persist": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
     "spec_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "spec_last_launch_count": (ctypes.c_int32, []),
@@ -160,6 +161,15 @@ def cycle(p: Params, base, target, U, W, last_token, draft, out, tau, p_draft, q
     _check(lib().spec_cycle(ctypes.byref(p.c()), _ptr(base), _ptr(target), _ptr(U), _ptr(W),
                             _ptr(last_token), _ptr(draft), _ptr(out), _ptr(tau), _ptr(p_draft),
                             _ptr(q_draft), _ptr(ws), _stream(stream)), "spec_cycle")
+
+
+def cycle_noalloc(p: Params, base, target, U, W, last_token, draft, out, tau, p_draft, q_draft,
+                  status_out=None, stream=None):
+    """spec_cycle on the library's built-in scratch array (no workspace)."""
+    _check(lib().spec_cycle_noalloc(ctypes.byref(p.c()), _ptr(base), _ptr(target), _ptr(U),
+                                    _ptr(W), _ptr(last_token), _ptr(draft), _ptr(out), _ptr(tau),
+                                    _ptr(p_draft), _ptr(q_draft), _ptr(status_out),
+                                    _stream(stream)), "spec_cycle_noalloc")
 
 
 def sync_status(ws, stream=None) -> int:

@@ -141,6 +141,24 @@ spec_status spec_cycle(const spec_params *p, const void *base, const void *targe
                        int32_t *tau, float *p_draft, float *q_draft, void *workspace,
                        spec_stream_t stream);
 
+/* spec_cycle without a workspace argument, for callers that cannot allocate
+ * device memory when they run a cycle (code whose allocations all belong to a
+ * framework pool, a host thread that must not call cudaMalloc because it
+ * synchronises the device, a plugin that only receives input and output
+ * buffers).  The pages have no counterpart: this is a deployment convenience.
+ * Scratch lives in a fixed 8 MiB device array inside the library, present on
+ * every GPU that loads it until the process exits; nothing is allocated per
+ * call.  Shapes whose spec_workspace_size exceeds 8 MiB are rejected with
+ * SPEC_ERR_WORKSPACE (and a message on stderr).  The first call on a device
+ * looks up the array's device address; make that first call before any stream
+ * capture.  All calls share the array: calls that overlap on the GPU race, so
+ * order them on one stream.  status_out (device int32, may be NULL) receives
+ * the device-side status of the call, stream-ordered after it. */
+spec_status spec_cycle_noalloc(const spec_params *p, const void *base, const void *target,
+                               const void *U, const void *W, const int32_t *last_token,
+                               int32_t *draft, int32_t *out, int32_t *tau, float *p_draft,
+                               float *q_draft, int32_t *status_out, spec_stream_t stream);
+
 /* Keep [ptr, ptr + bytes) resident in L2 for kernels later launched on
  * `stream` (a persisting access-policy window on the stream; the persisting
  * L2 carve-out of the calling process's context is raised to fit, up to the

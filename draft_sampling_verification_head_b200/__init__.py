@@ -46,7 +46,7 @@ class SpecParams(ctypes.Structure):
                 ("temperature", ctypes.c_float), ("greedy", ctypes.c_int32),
                 ("seed", ctypes.c_uint64), ("cycle", ctypes.c_uint64),
                 ("spin_limit", ctypes.c_uint64), ("flags", ctypes.c_uint32),
-                ("reserved", ctypes.c_uint32)]
+                ("row_offset", ctypes.c_uint32)]
 
 
 _lib = None
@@ -91,13 +91,15 @@ class Params:
     spin_limit: int = 0
     flags: int = 0
     draft_dtype: str | None = None
+    row_offset: int = 0  # global index of batch row 0 (Philox counter word 1)
 
     def c(self) -> SpecParams:
         dt = {"f32": SPEC_F32, "bf16": SPEC_BF16}
         return SpecParams(self.B, self.K, self.V, self.r, dt[self.dtype],
                           dt[self.draft_dtype or self.dtype], float(self.temperature),
                           1 if self.greedy else 0, self.seed & (2**64 - 1),
-                          self.cycle & (2**64 - 1), self.spin_limit, self.flags, 0)
+                          self.cycle & (2**64 - 1), self.spin_limit, self.flags,
+                          self.row_offset)
 
 
 def _ptr(t):

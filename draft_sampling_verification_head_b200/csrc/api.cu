@@ -32,6 +32,7 @@ spec_status check_params(const spec_params* p) {
   if (p->B < 1 || p->K < 1 || p->K > 1024 || p->V < 1 || p->r < 0 || p->r > 256)
     return SPEC_ERR_INVALID_ARG;
   if (p->dtype != SPEC_F32 && p->dtype != SPEC_BF16) return SPEC_ERR_INVALID_ARG;
+  if ((uint64_t)p->row_offset + (uint64_t)p->B > (uint64_t(1) << 31)) return SPEC_ERR_INVALID_ARG;
   if (!p->greedy && !(p->temperature > 0.f)) return SPEC_ERR_INVALID_ARG;
   if (p->V % 8 != 0) return SPEC_ERR_UNSUPPORTED;  // rows must start on 16-byte boundaries
   return SPEC_OK;
@@ -258,6 +259,7 @@ static spec_status run_cycle(const spec_params* p, int mode, const void* base, c
   L.temperature = p->temperature;
   L.seed = p->seed;
   L.cycle = p->cycle;
+  L.row0 = p->row_offset;
   L.spin = spin_of(p);
   L.trace = (p->flags & SPEC_FLAG_TRACE) != 0;
   cudaError_t e = launch_cycle(L, g, header_of(ws), body_of(ws), g.tc ? &tmW : nullptr, &tmBase,
@@ -306,19 +308,19 @@ spec_status spec_verify_block(const spec_params* p, const void* target, const vo
   uint8_t* body = body_of(ws);
   if (p->dtype == SPEC_BF16 && p->draft_dtype == SPEC_BF16)
     e = launch_verify((const __nv_bfloat16*)target, (const __nv_bfloat16*)draft_logits, draft, out,
-                      tau, p_draft, q_draft, B, K, V, p->temperature, gr, p->seed, p->cycle, body,
+                      tau, p_draft, q_draft, B, K, V, p->temperature, gr, p->seed, p->cycle, p->row_offset, body,
                       h, sms, st, &launches);
   else if (p->dtype == SPEC_BF16)
     e = launch_verify((const __nv_bfloat16*)target, (const float*)draft_logits, draft, out, tau,
-                      p_draft, q_draft, B, K, V, p->temperature, gr, p->seed, p->cycle, body, h,
+                      p_draft, q_draft, B, K, V, p->temperature, gr, p->seed, p->cycle, p->row_offset, body, h,
                       sms, st, &launches);
   else if (p->draft_dtype == SPEC_BF16)
     e = launch_verify((const float*)target, (const __nv_bfloat16*)draft_logits, draft, out, tau,
-                      p_draft, q_draft, B, K, V, p->temperature, gr, p->seed, p->cycle, body, h,
+                      p_draft, q_draft, B, K, V, p->temperature, gr, p->seed, p->cycle, p->row_offset, body, h,
                       sms, st, &launches);
   else
     e = launch_verify((const float*)target, (const float*)draft_logits, draft, out, tau, p_draft,
-                      q_draft, B, K, V, p->temperature, gr, p->seed, p->cycle, body, h, sms, st,
+                      q_draft, B, K, V, p->temperature, gr, p->seed, p->cycle, p->row_offset, body, h, sms, st,
                       &launches);
   g_last_launches = launches;
   return e == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;

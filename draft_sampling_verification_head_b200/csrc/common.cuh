@@ -27,7 +27,8 @@ struct WsHeader {
   uint32_t tok;         // tokens published in the current launch
   uint32_t exit_count;  // CTAs that finished the current launch
   uint32_t abort;       // nonzero once a CTA of the current launch gave up
-  uint32_t pad[56];
+  uint32_t rec;         // row records published in the current launch
+  uint32_t pad[55];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
@@ -41,6 +42,7 @@ enum ErrSite : int32_t {
   SITE_TOKEN_RANGE = 6,
   SITE_MBAR_BREADY = 7,
   SITE_MBAR_TFREE = 8,
+  SITE_REC_WAIT = 9,
 };
 
 SPEC_DEV void record_error(WsHeader* h, int32_t code, int32_t site, int32_t a, int32_t b) {

@@ -44,11 +44,12 @@ namespace {
 
 constexpr int kCH = 128;            // tokens per chunk (UMMA M)
 constexpr int kComputeThreads = 256;
-constexpr int kThreads = 320;       // 8 compute warps + TMA warp + MMA warp
+constexpr int kThreads = 352;       // 8 compute warps + W producer + MMA + base producer
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr int kNS = 8;              // W ring stages
-constexpr int kNBS = 2;             // base tile ring stages
+constexpr int kBaseWarp = 10;
+constexpr int kNS = 6;              // W ring stages
+constexpr int kNBS = 4;             // base tile ring stages
 constexpr int kMaxNC = 32;
 constexpr int kWStage = kCH * 64 * 2;  // 16 KB: 128 tokens x 64 rank, bf16
 constexpr int kMaxG = 160;          // CTAs a launch may use (>= SM count); partial-row stride
@@ -70,15 +71,16 @@ struct Args {
   float* q_draft;
   float* biased_out;
   WsHeader* hdr;
-  float2* dpart;     // [2][K+1][N][kMaxG]
-  float2* tpart;     // [2][K+1][N][kMaxG]
+  float4* dpart;     // [2][K+1][N][kMaxG]: (m, s, true max, 0) or (max, idx, max, 0)
+  float2* tpart;     // [2][K+1][N][kMaxG]: (m, s) or (max, idx)
   int32_t* tokens;   // [2][K][N]
   int32_t* accf;     // [2][K][N]
-  StopInfo* stopinfo;// [2][N]
+  struct Rec* rec;   // [2][K+2][N] row records
   uint64_t* trace;   // [K+2][kTracePhases] device timeline of CTA 0, or null
   int B, K, V, r, G, nc, nchunks, mode, greedy, ngroups;
   float k;           // log2(e) / T (1 in greedy mode)
   uint64_t seed, cycle, spin;
+  uint32_t row0;  // global index of batch row 0 (Philox counter word 1)
 };
 
 template <int N>
@@ -97,10 +99,50 @@ struct Ctl {
   int32_t tok[N];
   float M[N], S[N];     // global draft stats of the current step
   float zM[N], zS[N];   // draft stats of the stop row
-  float Mt[N], St[N];   // target stats (row i during a step, stop row / row K at the end)
-  int16_t wlist[8][N];  // owned rows per compute warp
-  int32_t wcount[8];
+  float Mt[N], St[N];   // target stats of row i during a step
+  float fMt[N], fSt[N]; // target stats of the final row (stop row or row K)
+  float ref[N];         // per-row reference of the fast path (previous step's max)
+  float cmax[4][N];     // true max per row and tensor-memory quadrant
+  int32_t redo;
 };
+
+// One record per batch row and reduction, written by the row's reducer.
+struct alignas(16) Rec {
+  float M, S;       // scale (reference) and total of the draw's distribution
+  float Mx;         // true max of z this step (the next step's reference)
+  float Mt, St;     // target row statistics
+  float trem;       // inverse-CDF target inside the owner CTA's slice (inf: last mass)
+  int32_t owner;    // CTA that owns the draw
+  int32_t token;    // greedy: arg-max draft token
+  int32_t acc;      // greedy: accept outcome
+  int32_t flags;    // bit 0: redo the step exactly; bit 1: final draw uses p
+  int32_t tam;      // greedy: target arg-max
+  int32_t pad;
+};
+static_assert(sizeof(Rec) == 48, "records are three 16-byte words");
+
+SPEC_DEV void store_rec(Rec* dst, const Rec& r) {
+  const float4* s4 = reinterpret_cast<const float4*>(&r);
+  float4* d4 = reinterpret_cast<float4*>(dst);
+  d4[0] = s4[0];
+  d4[1] = s4[1];
+  d4[2] = s4[2];
+}
+SPEC_DEV Rec load_rec(const Rec* src) {
+  Rec r;
+  float4* d4 = reinterpret_cast<float4*>(&r);
+  const float4* s4 = reinterpret_cast<const float4*>(src);
+  d4[0] = __ldcg(s4);
+  d4[1] = __ldcg(s4 + 1);
+  d4[2] = __ldcg(s4 + 2);
+  return r;
+}
+
+// Shared region for per-bucket statistics, reused to stage owned rows' values.
+__host__ __device__ inline size_t bucket_region_bytes(int nc, int N) {
+  const size_t b = (size_t)nc * 4 * N * sizeof(float2), z = (size_t)N * 32 * sizeof(float);
+  return b > z ? b : z;
+}
 
 SPEC_DEV void named_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
@@ -222,6 +264,38 @@ SPEC_DEV void bfly_sum2(float (&a)[NCOL], float (&c)[NCOL], int lane) {
   }
 }
 
+template <int NCOL>
+SPEC_DEV void bfly_sum1(float (&a)[NCOL], int lane) {
+#pragma unroll
+  for (int h = NCOL / 2, off = 16; h >= 1; h >>= 1, off >>= 1) {
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int j = 0; j < h; ++j) {
+      const float sa = up ? a[j] : a[j + h];
+      const float ka = up ? a[j + h] : a[j];
+      a[j] = ka + __shfl_xor_sync(FULL, sa, off);
+    }
+  }
+#pragma unroll
+  for (int off = 16 / NCOL; off >= 1; off >>= 1) a[0] += __shfl_xor_sync(FULL, a[0], off);
+}
+
+template <int NCOL>
+SPEC_DEV void bfly_max1(float (&a)[NCOL], int lane) {
+#pragma unroll
+  for (int h = NCOL / 2, off = 16; h >= 1; h >>= 1, off >>= 1) {
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int j = 0; j < h; ++j) {
+      const float sa = up ? a[j] : a[j + h];
+      const float ka = up ? a[j + h] : a[j];
+      a[j] = fmaxf(ka, __shfl_xor_sync(FULL, sa, off));
+    }
+  }
+#pragma unroll
+  for (int off = 16 / NCOL; off >= 1; off >>= 1) a[0] = fmaxf(a[0], __shfl_xor_sync(FULL, a[0], off));
+}
+
 // tcgen05.ld of NCOL consecutive columns (NCOL multiple of 8)
 template <int NCOL>
 SPEC_DEV void tmem_ld_cols(uint32_t taddr, float (&v)[NCOL]) {
@@ -277,8 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
   T* sBase = reinterpret_cast<T*>(sU + ((u_bytes + 1023) & ~size_t(1023)));  // kNBS x N x 128
   const size_t base_bytes = (size_t)kNBS * N * kCH * sizeof(T);
   float2* sBucket = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(sBase) + base_bytes);
+  float* zbuf = reinterpret_cast<float*>(sBucket);  // owner staging, after the bucket walk
   Ctl<N>* ctl = reinterpret_cast<Ctl<N>*>(reinterpret_cast<uint8_t*>(sBucket) +
-                                          (size_t)a.nc * 4 * N * sizeof(float2));
+                                          bucket_region_bytes(a.nc, N));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cta = blockIdx.x;
@@ -325,50 +400,35 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
   const uint32_t taddr = ctl->tmem_slot;
 
   // =========================================================================
-  // TMA producer: W ring (tensor-core path) and base tiles, in consumption order
+  // TMA producers, each in its own consumption order: the W ring (tensor-core
+  // path) on one warp, the base logit tiles on another, so neither stream
+  // waits behind the other.
   // =========================================================================
   if (warp == kProducerWarp) {
-    if (lane == 0) {
-      const uint64_t polW = policy_evict_last(), polB = policy_evict_first();
-      if (TC) tma_prefetch_desc(&a.tmW);
-      tma_prefetch_desc(&a.tmBase);
-      uint32_t Lw = 0, Lb = 0;
+    if (TC && lane == 0) {
+      const uint64_t polW = policy_evict_last();
+      tma_prefetch_desc(&a.tmW);
+      uint32_t Lw = 0;
       bool ok = true;
       for (int g = 0; g < a.ngroups && ok; ++g) {
         for (int s = 0; s < nsteps && ok; ++s) {
           for (int cl = 0; cl < ncc && ok; ++cl) {
             const int v0 = (chunk0 + cl) * kCH;
-            if (TC) {
-              for (int kb = 0; kb < nkb; ++kb) {
-                const uint32_t slot = Lw % kNS;
-                if (Lw >= kNS &&
-                    !mbar_wait_bounded(&ctl->wempty[slot], ((Lw / kNS) - 1) & 1, a.spin,
-                                       &hdr->abort)) {
-                  record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_FULL, cta, 100 + s);
-                  ok = false;
-                  break;
-                }
-                mbar_arrive_expect_tx(&ctl->wfull[slot], kWStage);
-                tma_load_2d(sW + (size_t)slot * kWStage, &a.tmW, &ctl->wfull[slot], v0, kb * 64,
-                            polW);
-                tma_load_2d(sW + (size_t)slot * kWStage + kWStage / 2, &a.tmW,
-                            &ctl->wfull[slot], v0 + 64, kb * 64, polW);
-                ++Lw;
-              }
-            }
-            if (ok && s < K) {
-              const uint32_t slot = Lb % kNBS;
-              if (Lb >= kNBS &&
-                  !mbar_wait_bounded(&ctl->bempty[slot], ((Lb / kNBS) - 1) & 1, a.spin,
+            for (int kb = 0; kb < nkb; ++kb) {
+              const uint32_t slot = Lw % kNS;
+              if (Lw >= kNS &&
+                  !mbar_wait_bounded(&ctl->wempty[slot], ((Lw / kNS) - 1) & 1, a.spin,
                                      &hdr->abort)) {
-                record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_BASE, cta, s);
+                record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_FULL, cta, 100 + s);
                 ok = false;
                 break;
               }
-              mbar_arrive_expect_tx(&ctl->bfull[slot], (uint32_t)(N * kCH * sizeof(T)));
-              tma_load_3d(sBase + (size_t)slot * N * kCH, &a.tmBase, &ctl->bfull[slot], v0, s,
-                          g * N, polB);
-              ++Lb;
+              mbar_arrive_expect_tx(&ctl->wfull[slot], kWStage);
+              tma_load_2d(sW + (size_t)slot * kWStage, &a.tmW, &ctl->wfull[slot], v0, kb * 64,
+                          polW);
+              tma_load_2d(sW + (size_t)slot * kWStage + kWStage / 2, &a.tmW, &ctl->wfull[slot],
+                          v0 + 64, kb * 64, polW);
+              ++Lw;
             }
           }
         }
@@ -376,6 +436,31 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
       // drain: the most recent load on every slot must have landed
       for (uint32_t L = (Lw > kNS ? Lw - kNS : 0); L < Lw; ++L)
         mbar_drain(&ctl->wfull[L % kNS], (L / kNS) & 1);
+    }
+  } else if (warp == kBaseWarp) {
+    if (lane == 0) {
+      const uint64_t polB = policy_evict_first();
+      tma_prefetch_desc(&a.tmBase);
+      uint32_t Lb = 0;
+      bool ok = true;
+      for (int g = 0; g < a.ngroups && ok; ++g) {
+        for (int s = 0; s < K && ok; ++s) {
+          for (int cl = 0; cl < ncc; ++cl) {
+            const uint32_t slot = Lb % kNBS;
+            if (Lb >= kNBS &&
+                !mbar_wait_bounded(&ctl->bempty[slot], ((Lb / kNBS) - 1) & 1, a.spin,
+                                   &hdr->abort)) {
+              record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_BASE, cta, s);
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&ctl->bfull[slot], (uint32_t)(N * kCH * sizeof(T)));
+            tma_load_3d(sBase + (size_t)slot * N * kCH, &a.tmBase, &ctl->bfull[slot],
+                        (chunk0 + cl) * kCH, s, g * N, polB);
+            ++Lb;
+          }
+        }
+      }
       for (uint32_t L = (Lb > kNBS ? Lb - kNBS : 0); L < Lb; ++L)
         mbar_drain(&ctl->bfull[L % kNBS], (L / kNBS) & 1);
     }
@@ -440,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
     const int q4 = warp & 3;         // tensor-memory lane quadrant
     const int n0 = (warp >> 2) * NCOL;  // first column (batch row) of this warp
     uint32_t step_ctr = 0, Lb = 0;
-    uint32_t nbar = 0, tok_expected = 0;
+    uint32_t nbar = 0, tok_expected = 0, rec_expected = 0;
     // Failures are folded into the CTA-wide flag ctl->abort_local; it is only
     // read right after a named barrier, so every compute thread takes the same
     // branch (a waiter that gives up keeps executing until that point).
@@ -570,101 +655,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
       }
     };
 
-    // ---- combine of the G per-CTA partials of one batch row: TPB threads per
-    // row, each holding a contiguous slice of the partials in registers (all
-    // loads in flight together).  Identical arithmetic in every CTA.
-    constexpr int MAXC = kMaxG / TPB;  // partials per thread (even: 16-byte loads)
-    static_assert(MAXC % 2 == 0, "partial slices are read as float4");
+    // ---- CTA partial per batch row is formed by TPB threads per row
     const int grp_n = tid / TPB, grp_sub = tid % TPB;
-    const int c_lo = grp_sub * MAXC;
-    const int c_hi = min(G, c_lo + MAXC);
-    // Unconditional 16-byte loads over the padded row (entries past G or of
-    // rows not in use are replaced afterwards), so all are in flight together.
-    auto load_slice = [&](const float2* pp, bool on, float2 (&reg)[MAXC], float2 dflt) {
-      const float4* p4 = reinterpret_cast<const float4*>(pp + c_lo);
-#pragma unroll
-      for (int j = 0; j < MAXC / 2; ++j) {
-        const float4 q = __ldcg(p4 + j);
-        reg[2 * j] = make_float2(q.x, q.y);
-        reg[2 * j + 1] = make_float2(q.z, q.w);
-      }
-#pragma unroll
-      for (int j = 0; j < MAXC; ++j)
-        if (!(on && c_lo + j < c_hi)) reg[j] = dflt;
-    };
-    // (m, s) partials -> global M, S (valid in every thread of the group)
-    auto group_ms = [&](const float2 (&reg)[MAXC], float& M, float& S) {
-      float m = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < MAXC; ++j) m = fmaxf(m, reg[j].x);
-#pragma unroll
-      for (int off = TPB / 2; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
-      float loc = 0.f;
-#pragma unroll
-      for (int j = 0; j < MAXC; ++j)
-        if (reg[j].y > 0.f) loc += reg[j].y * exp2f((reg[j].x - m) * k);
-      float sum = loc;
-#pragma unroll
-      for (int off = TPB / 2; off >= 1; off >>= 1) sum += __shfl_xor_sync(FULL, sum, off);
-      M = m;
-      S = sum;
-    };
-    auto group_amax = [&](const float2 (&reg)[MAXC], float& av, int32_t& ai) {
-      av = -INFINITY;
-      ai = 0x7fffffff;
-#pragma unroll
-      for (int j = 0; j < MAXC; ++j) amax_combine(av, ai, reg[j].x, __float_as_int(reg[j].y));
-#pragma unroll
-      for (int off = TPB / 2; off >= 1; off >>= 1) {
-        const float a2 = __shfl_xor_sync(FULL, av, off);
-        const int32_t i2 = __shfl_xor_sync(FULL, ai, off);
-        amax_combine(av, ai, a2, i2);
-      }
-    };
-    // Inverse-CDF owner among the G CTAs for weights w_c (given by wfun(j)),
-    // scanned in ascending c; returns true in the one thread whose slice holds
-    // the owner, with the owner index and the mass before it.
-    // weight of a partial: wmode 0 -> s * exp2((m - M) k) (softmax partials),
-    // 1 -> .x (residual mass), 2 -> .y (target mass)
-    auto pweight = [&](const float2& p, int wmode, float M) {
-      if (wmode == 0) return p.y > 0.f ? p.y * exp2f((p.x - M) * k) : 0.f;
-      return wmode == 1 ? p.x : p.y;
-    };
-    auto group_owner = [&](const float2 (&reg)[MAXC], int wmode, float M, float tgt, int& own,
-                           float& before, bool& fallback) {
-      float loc = 0.f;
-#pragma unroll
-      for (int j = 0; j < MAXC; ++j) loc += pweight(reg[j], wmode, M);
-      float incl = loc;
-#pragma unroll
-      for (int o = 1; o < TPB; o <<= 1) {
-        const float y = __shfl_up_sync(FULL, incl, o, TPB);
-        if (grp_sub >= o) incl += y;
-      }
-      float cum = incl - loc;
-      int found = 0x7fffffff, lastpos = -1;
-      before = 0.f;
-#pragma unroll
-      for (int j = 0; j < MAXC; ++j) {
-        if (c_lo + j >= c_hi) continue;
-        const float wj = pweight(reg[j], wmode, M);
-        if (wj > 0.f) lastpos = c_lo + j;
-        if (found == 0x7fffffff && cum + wj > tgt) {
-          found = c_lo + j;
-          before = cum;
-        }
-        cum += wj;
-      }
-      int o2 = found;
-#pragma unroll
-      for (int off = TPB / 2; off >= 1; off >>= 1) o2 = min(o2, __shfl_xor_sync(FULL, o2, off));
-      int lp = lastpos;
-#pragma unroll
-      for (int off = TPB / 2; off >= 1; off >>= 1) lp = max(lp, __shfl_xor_sync(FULL, lp, off));
-      fallback = o2 == 0x7fffffff;
-      own = fallback ? lp : o2;
-      return fallback ? (lastpos == own && own >= 0) : (found == own);
-    };
 
     // Gather U[prev] rows (ctl->prev) into the B operand.
     auto gather_u = [&](int nb_g) {
@@ -736,9 +728,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
       return pos ? 31 - __clz(pos) : 0;
     };
 
-    // Bucket walk for every owned row (one thread each), then per-warp work
-    // lists: a row goes to one of the two warps of its bucket's quadrant.
-    // `mass(n, cl, q)` gives the bucket weight in the owner's scale.
     // fin = false: softmax buckets (m, s) in the scale of ctl->M[n];
     // fin = true: residual / target mass buckets, chosen by ctl->S[n] != 0.
     auto bucket_mass = [&](int n, int cl, int q, bool fin) {
@@ -746,10 +735,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
       if (!fin) return p.y > 0.f ? p.y * exp2f((p.x - ctl->M[n]) * k) : 0.f;
       return ctl->S[n] != 0.f ? p.y : p.x;
     };
+    // Bucket walk for every owned row (one warp per row, lanes = buckets),
+    // then per-warp work lists: a row goes to one of the two warps of its
+    // bucket's quadrant.
     auto walk_and_assign = [&](bool fin) {
       const int n_owned = ctl->n_owned;
       const int nbk = ncc * 4;  // buckets in ascending token order
-      for (int o = warp; o < n_owned; o += 8) {  // one warp per owned row
+      for (int o = warp; o < n_owned; o += 8) {
         const int n = ctl->owned[o];
         const float tin = ctl->obtarget[o];
         float carry = 0.f;
@@ -784,18 +776,204 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
         }
       }
       named_sync();
-      if (tid < 4) {
-        int c0 = 0, c1 = 0, alt = 0;
-        for (int o = 0; o < n_owned; ++o) {
-          if ((ctl->obucket[o] & 3) != tid) continue;
-          if (alt) ctl->wlist[tid + 4][c1++] = (int16_t)o;
-          else ctl->wlist[tid][c0++] = (int16_t)o;
-          alt ^= 1;
+      // Stage the chosen bucket of every owned row (32 values from tensor
+      // memory, reachable only from the warps of that lane quadrant) into
+      // shared memory, so that any warp can then scan any owned row.
+      {
+        tc_fence_after();
+        int mine = 0;
+        for (int o0 = 0; o0 < n_owned;) {
+          int oo[kOwnBatch];
+          float vv[kOwnBatch];
+          int got = 0;
+          for (; o0 < n_owned && got < kOwnBatch; ++o0) {
+            if ((ctl->obucket[o0] & 3) != q4) continue;
+            if (((mine++) & 1) != (warp >> 2)) continue;
+            oo[got++] = o0;
+          }
+#pragma unroll
+          for (int j = 0; j < kOwnBatch; ++j) {
+            vv[j] = 0.f;
+            if (j >= got) continue;
+            const int cl = ctl->obucket[oo[j]] >> 2, n = ctl->owned[oo[j]];
+            tmem_ld1(taddr + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(cl * N + n), &vv[j]);
+          }
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < kOwnBatch; ++j)
+            if (j < got) zbuf[oo[j] * 32 + lane] = vv[j];
         }
-        ctl->wcount[tid] = c0;
-        ctl->wcount[tid + 4] = c1;
       }
       named_sync();
+    };
+
+    // ---- row reducers.  Row n of a group is combined by one warp of CTA
+    // n % G; lanes hold E consecutive per-CTA partials each, so a warp prefix
+    // sum walks the CTAs in ascending token order.  The reducer alone decides
+    // the owner CTA of the row's inverse-CDF draw and publishes a record.
+    //  kind 0: draft step i -- stochastic: scale, total, owner, residual target,
+    //          true max; greedy: the arg-max token; plus target row i
+    //          statistics (or arg-max and the accept outcome) for live rows;
+    //  kind 1: target row K statistics (or arg-max) for rows that accepted all;
+    //  kind 2: final residual / bonus masses -- owner of the last draw.
+    constexpr int E = (kMaxG + 31) / 32;
+    auto reduce_rows = [&](int kind, int g, int par, int i, int nb_g, bool fast) {
+      int mine = 0, local = 0;
+      for (int n = cta; n < nb_g; n += G, ++local) {
+        ++mine;
+        if ((local & 7) != warp) continue;  // warp-uniform
+        const int b = g * N + n;
+        const int c0 = lane * E;
+        Rec rc;
+        rc.M = 0.f; rc.S = 1.f; rc.Mx = 0.f; rc.Mt = 0.f; rc.St = 1.f; rc.trem = INFINITY;
+        rc.owner = 0; rc.token = 0; rc.acc = 1; rc.flags = 0; rc.tam = 0; rc.pad = 0;
+        if (kind == 0 || kind == 2) {
+          const int slot = kind == 0 ? i : K;
+          const float4* pp = a.dpart + ((((int64_t)par * (K + 1) + slot) * N + n) * kMaxG + c0);
+          float4 v[E];
+#pragma unroll
+          for (int t = 0; t < E; ++t) v[t] = __ldcg(pp + t);
+          if (kind == 0 && a.greedy) {
+            float av = -INFINITY;
+            int32_t ai = 0x7fffffff;
+#pragma unroll
+            for (int t = 0; t < E; ++t)
+              if (c0 + t < G) amax_combine(av, ai, v[t].x, __float_as_int(v[t].y));
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) {
+              const float a2 = __shfl_xor_sync(FULL, av, off);
+              const int32_t i2 = __shfl_xor_sync(FULL, ai, off);
+              amax_combine(av, ai, a2, i2);
+            }
+            rc.token = ai;
+          } else {
+            float w[E];
+            float M = -INFINITY, mx = -INFINITY;
+            bool use_p = false;
+            if (kind == 0) {
+#pragma unroll
+              for (int t = 0; t < E; ++t)
+                if (c0 + t < G) {
+                  M = fmaxf(M, v[t].x);
+                  mx = fmaxf(mx, v[t].z);
+                }
+#pragma unroll
+              for (int off = 16; off >= 1; off >>= 1) {
+                M = fmaxf(M, __shfl_xor_sync(FULL, M, off));
+                mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, off));
+              }
+#pragma unroll
+              for (int t = 0; t < E; ++t)
+                w[t] = (c0 + t < G && v[t].y > 0.f) ? v[t].y * exp2f((v[t].x - M) * k) : 0.f;
+            } else {
+              float rt = 0.f, pt = 0.f;
+#pragma unroll
+              for (int t = 0; t < E; ++t)
+                if (c0 + t < G) {
+                  rt += v[t].x;
+                  pt += v[t].y;
+                }
+              rt = warp_sum(rt);
+              use_p = !(rt > 0.f);
+#pragma unroll
+              for (int t = 0; t < E; ++t) w[t] = c0 + t < G ? (use_p ? v[t].y : v[t].x) : 0.f;
+            }
+            float loc = 0.f;
+#pragma unroll
+            for (int t = 0; t < E; ++t) loc += w[t];
+            float incl = loc;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+              const float y = __shfl_up_sync(FULL, incl, off);
+              if (lane >= off) incl += y;
+            }
+            const float total = __shfl_sync(FULL, incl, 31);
+            const int row = kind == 0 ? i : (ctl->alive[n] ? K : ctl->stoprow[n]);
+            const float u = philox_uniform(a.seed, a.cycle, a.row0 + (uint32_t)b, (uint32_t)row,
+                                           kind == 0 ? TAG_DRAFT : TAG_RESAMPLE);
+            const float tgt = u * total;
+            float cum = incl - loc, before = 0.f;
+            int found = 0x7fffffff, lastpos = -1;
+#pragma unroll
+            for (int t = 0; t < E; ++t) {
+              if (w[t] > 0.f) lastpos = c0 + t;
+              if (found == 0x7fffffff && w[t] > 0.f && cum + w[t] > tgt) {
+                found = c0 + t;
+                before = cum;
+              }
+              cum += w[t];
+            }
+            int own = found;
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) own = min(own, __shfl_xor_sync(FULL, own, off));
+            int lp = lastpos;
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) lp = max(lp, __shfl_xor_sync(FULL, lp, off));
+            const bool fb = own == 0x7fffffff;
+            const float bown = __shfl_sync(FULL, before, fb ? 0 : own / E);
+            rc.owner = fb ? max(lp, 0) : own;
+            rc.trem = fb ? INFINITY : tgt - bown;
+            rc.M = M;
+            rc.S = total;
+            rc.Mx = mx;
+            if (kind == 0 && fast && (fabsf(mx - M) * k > 64.f || !(total > 0.f))) rc.flags |= 1;
+            if (kind == 2 && use_p) rc.flags |= 2;
+          }
+        }
+        const bool live = ctl->alive[n] != 0;
+        if ((kind == 0 && a.mode == MODE_CYCLE && live) || (kind == 1 && live)) {
+          const int row = kind == 0 ? i : K;
+          const float2* tp = a.tpart + ((((int64_t)par * (K + 1) + row) * N + n) * kMaxG + c0);
+          float2 tv[E];
+#pragma unroll
+          for (int t = 0; t < E; ++t) tv[t] = __ldcg(tp + t);
+          if (a.greedy) {
+            float av = -INFINITY;
+            int32_t ai = 0x7fffffff;
+#pragma unroll
+            for (int t = 0; t < E; ++t)
+              if (c0 + t < G) amax_combine(av, ai, tv[t].x, __float_as_int(tv[t].y));
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) {
+              const float a2 = __shfl_xor_sync(FULL, av, off);
+              const int32_t i2 = __shfl_xor_sync(FULL, ai, off);
+              amax_combine(av, ai, a2, i2);
+            }
+            rc.tam = ai;
+            if (kind == 0) rc.acc = ai == rc.token ? 1 : 0;
+          } else {
+            float Mt = -INFINITY;
+#pragma unroll
+            for (int t = 0; t < E; ++t)
+              if (c0 + t < G) Mt = fmaxf(Mt, tv[t].x);
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) Mt = fmaxf(Mt, __shfl_xor_sync(FULL, Mt, off));
+            float st = 0.f;
+#pragma unroll
+            for (int t = 0; t < E; ++t)
+              if (c0 + t < G && tv[t].y > 0.f) st += tv[t].y * exp2f((tv[t].x - Mt) * k);
+            rc.Mt = Mt;
+            rc.St = warp_sum(st);
+          }
+        }
+        if (lane == 0) store_rec(a.rec + ((int64_t)par * (K + 2) + (kind == 0 ? i : (kind == 1 ? K : K + 1))) * N + n, rc);
+      }
+      return mine;
+    };
+    // publish this CTA's records and wait until every row's record exists
+    auto records_hop = [&](int mine, int nb_g) {
+      named_sync();
+      if (tid == 0) {
+        __threadfence();
+        if (mine) red_release_add_u32(&hdr->rec, (uint32_t)mine);
+        rec_expected += (uint32_t)nb_g;
+        if (!grid_wait_count(hdr, &hdr->rec, rec_expected, a.spin, SITE_REC_WAIT) ||
+            ld_volatile_u32(&hdr->abort))
+          ctl->abort_local = 1;
+        __threadfence();
+      }
+      named_sync();
+      return ctl->abort_local == 0;
     };
 
     for (int g = 0; g < a.ngroups && !failed; ++g) {
@@ -804,6 +982,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
       for (int n = tid; n < N; n += kComputeThreads) {
         ctl->alive[n] = n < nb_g ? 1 : 0;
         ctl->stoprow[n] = K;
+        ctl->ref[n] = 0.f;
       }
       if (cta == 0 && a.mode == MODE_CYCLE) {
         for (int idx = tid; idx < nb_g * K; idx += kComputeThreads) {
@@ -844,170 +1023,167 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
                            (uint32_t)((vslice_hi - vslice_lo) * sizeof(T)));
         mark(g, i, 1);
 
-        // ---------------- epilogue: z = base + bias, bucket statistics
-        uint64_t t_wait = 0;
-        for (int cl = 0; cl < ncc; ++cl) {
-          float d[NCOL];
-          const uint64_t t_w0 = trace ? globaltimer_ns() : 0;
-          bias_tile(cl, d);
-          if (trace) t_wait += globaltimer_ns() - t_w0;
-          const uint32_t bslot = Lb % kNBS;
-          if (!mbar_wait_bounded(&ctl->bfull[bslot], (Lb / kNBS) & 1, a.spin, &hdr->abort))
-            soft_fail(SPEC_ERR_TIMEOUT, SITE_MBAR_BASE, cta, i);
-          const T* bt = sBase + (size_t)bslot * N * kCH;
-          const int vl = q4 * 32 + lane;
-          const int v = (chunk0 + cl) * kCH + vl;
-          const bool valid = v < V;
+        // From step 1 on the softmax partials share a per-row reference (the
+        // previous step's true max), so bucket statistics are plain sums.
+        bool fast = !a.greedy && i > 0;
+        for (int attempt = 0; attempt < 2; ++attempt) {
+          // ---------------- epilogue: z = base + bias, bucket statistics
+          uint64_t t_wait = 0;
+          float rmax[NCOL];
 #pragma unroll
-          for (int j = 0; j < NCOL; ++j)
-            d[j] = valid ? d[j] + to_f<T>(bt[(n0 + j) * kCH + vl]) : -INFINITY;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&ctl->bempty[bslot]);
-          ++Lb;
-          // z replaces the bias in tensor memory: the owner scan reads it back
-          if (!a.greedy)
-            tmem_st_cols<NCOL>(taddr + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(cl * N + n0), d);
-          if (a.biased_out && valid) {
+          for (int j = 0; j < NCOL; ++j) rmax[j] = -INFINITY;
+          for (int cl = 0; cl < ncc; ++cl) {
+            float d[NCOL];
+            const int vl = q4 * 32 + lane;
+            const int v = (chunk0 + cl) * kCH + vl;
+            const bool valid = v < V;
+            const uint32_t tcol = taddr + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(cl * N + n0);
+            if (attempt == 0) {
+              const uint64_t t_w0 = trace ? globaltimer_ns() : 0;
+              bias_tile(cl, d);
+              if (trace) t_wait += globaltimer_ns() - t_w0;
+              const uint32_t bslot = Lb % kNBS;
+              if (!mbar_wait_bounded(&ctl->bfull[bslot], (Lb / kNBS) & 1, a.spin, &hdr->abort))
+                soft_fail(SPEC_ERR_TIMEOUT, SITE_MBAR_BASE, cta, i);
+              const T* bt = sBase + (size_t)bslot * N * kCH;
 #pragma unroll
-            for (int j = 0; j < NCOL; ++j) {
-              const int b = g * N + n0 + j;
-              if (n0 + j < nb_g) a.biased_out[((int64_t)b * K + i) * V + v] = d[j];
+              for (int j = 0; j < NCOL; ++j)
+                d[j] = valid ? d[j] + to_f<T>(bt[(n0 + j) * kCH + vl]) : -INFINITY;
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&ctl->bempty[bslot]);
+              ++Lb;
+              if (a.biased_out && valid) {
+#pragma unroll
+                for (int j = 0; j < NCOL; ++j) {
+                  const int b = g * N + n0 + j;
+                  if (n0 + j < nb_g) a.biased_out[((int64_t)b * K + i) * V + v] = d[j];
+                }
+              }
+              // z replaces the bias in tensor memory: owner scans (and a redo) read it
+              if (!a.greedy) tmem_st_cols<NCOL>(tcol, d);
+            } else {
+              tmem_ld_cols<NCOL>(tcol, d);  // z of this step, kept in tensor memory
+            }
+            float2* bk = sBucket + ((size_t)cl * 4 + q4) * N;
+            constexpr int REP = 32 / NCOL;
+            if (a.greedy) {
+              int32_t ix[NCOL];
+#pragma unroll
+              for (int j = 0; j < NCOL; ++j) ix[j] = valid ? v : 0x7fffffff;
+              bfly_amax<NCOL>(d, ix, lane);
+              if ((lane & (REP - 1)) == 0) bk[n0 + lane / REP] = make_float2(d[0], __int_as_float(ix[0]));
+            } else if (fast) {
+#pragma unroll
+              for (int j = 0; j < NCOL; ++j) {
+                rmax[j] = fmaxf(rmax[j], d[j]);
+                d[j] = valid ? exp2f((d[j] - ctl->ref[n0 + j]) * k) : 0.f;
+              }
+              bfly_sum1<NCOL>(d, lane);
+              if ((lane & (REP - 1)) == 0)
+                bk[n0 + lane / REP] = make_float2(ctl->ref[n0 + lane / REP], d[0]);
+            } else {
+              float s[NCOL];
+#pragma unroll
+              for (int j = 0; j < NCOL; ++j) s[j] = valid ? 1.f : 0.f;
+              bfly_ms<NCOL>(d, s, k, lane);
+              if ((lane & (REP - 1)) == 0) bk[n0 + lane / REP] = make_float2(d[0], s[0]);
             }
           }
-          float2* bk = sBucket + ((size_t)cl * 4 + q4) * N;
-          if (a.greedy) {
-            int32_t ix[NCOL];
-#pragma unroll
-            for (int j = 0; j < NCOL; ++j) ix[j] = valid ? v : 0x7fffffff;
-            bfly_amax<NCOL>(d, ix, lane);
-            if ((lane & (32 / NCOL - 1)) == 0)
-              bk[n0 + lane / (32 / NCOL)] = make_float2(d[0], __int_as_float(ix[0]));
-          } else {
-            float s[NCOL];
-#pragma unroll
-            for (int j = 0; j < NCOL; ++j) s[j] = valid ? 1.f : 0.f;
-            bfly_ms<NCOL>(d, s, k, lane);
-            if ((lane & (32 / NCOL - 1)) == 0) bk[n0 + lane / (32 / NCOL)] = make_float2(d[0], s[0]);
+          if (fast) {  // true max of z per row over this warp's tokens
+            bfly_max1<NCOL>(rmax, lane);
+            if ((lane & (32 / NCOL - 1)) == 0) ctl->cmax[q4][n0 + lane / (32 / NCOL)] = rmax[0];
           }
-        }
-        tc_fence_before();  // z stores above are read by other warps after the barrier
-        named_sync();
-        tc_fence_after();
-        mark(g, i, 2);
-        if (trace && g == 0) trace[(size_t)i * kTracePhases + 11] = t_wait;
-        // ---------------- CTA partial per batch row (TPB threads per row)
-        {
-          const int n = grp_n;
-          float m = -INFINITY, s = 0.f;
-          int32_t ai = 0x7fffffff;
-          for (int bk = grp_sub; bk < ncc * 4; bk += TPB) {
-            const float2 p = sBucket[(size_t)bk * N + n];
-            if (a.greedy)
-              amax_combine(m, ai, p.x, __float_as_int(p.y));
-            else
-              ms_combine(m, s, p.x, p.y, k);
-          }
+          tc_fence_before();  // z stores above are read by other warps after the barrier
+          named_sync();
+          tc_fence_after();
+          mark(g, i, 2);
+          if (trace && g == 0) trace[(size_t)i * kTracePhases + 11] = t_wait;
+          // ---------------- CTA partial per batch row (TPB threads per row)
+          {
+            const int n = grp_n;
+            float m = -INFINITY, s = 0.f;
+            int32_t ai = 0x7fffffff;
+            for (int bk = grp_sub; bk < ncc * 4; bk += TPB) {
+              const float2 p = sBucket[(size_t)bk * N + n];
+              if (a.greedy)
+                amax_combine(m, ai, p.x, __float_as_int(p.y));
+              else
+                ms_combine(m, s, p.x, p.y, k);
+            }
 #pragma unroll
-          for (int off = TPB / 2; off >= 1; off >>= 1) {
-            const float m2 = __shfl_xor_sync(FULL, m, off), s2 = __shfl_xor_sync(FULL, s, off);
-            const int32_t i2 = __shfl_xor_sync(FULL, ai, off);
-            if (a.greedy)
-              amax_combine(m, ai, m2, i2);
-            else
-              ms_combine(m, s, m2, s2, k);
+            for (int off = TPB / 2; off >= 1; off >>= 1) {
+              const float m2 = __shfl_xor_sync(FULL, m, off), s2 = __shfl_xor_sync(FULL, s, off);
+              const int32_t i2 = __shfl_xor_sync(FULL, ai, off);
+              if (a.greedy)
+                amax_combine(m, ai, m2, i2);
+              else
+                ms_combine(m, s, m2, s2, k);
+            }
+            if (grp_sub == 0) {
+              float tmax = m;
+              if (fast)
+                tmax = fmaxf(fmaxf(ctl->cmax[0][n], ctl->cmax[1][n]),
+                             fmaxf(ctl->cmax[2][n], ctl->cmax[3][n]));
+              a.dpart[(((int64_t)par * (K + 1) + i) * N + n) * kMaxG + cta] =
+                  a.greedy ? make_float4(m, __int_as_float(ai), m, 0.f) : make_float4(m, s, tmax, 0.f);
+            }
           }
-          if (grp_sub == 0)
-            a.dpart[(((int64_t)par * (K + 1) + i) * N + n) * kMaxG + cta] =
-                a.greedy ? make_float2(m, __int_as_float(ai)) : make_float2(m, s);
-        }
-        grid_arrive();
-        mark(g, i, 3);
-        // background while the barrier completes: next target row, rows alive so far
-        if (a.mode == MODE_CYCLE) target_row_stats(g, par, i + 1, nb_g);
-        mark(g, i, 4);
-        if (!grid_wait()) {
-          failed = true;
-          break;
-        }
-        mark(g, i, 5);
-
-        // ---------------- combine partials: every CTA, same order
-        if (tid == 0) ctl->n_owned = 0;
-        named_sync();
-        {
-          const int n = grp_n;
-          const bool row_on = n < nb_g;
-          float2 reg[MAXC];
-          load_slice(a.dpart + (((int64_t)par * (K + 1) + i) * N + n) * kMaxG, row_on, reg,
-                     a.greedy ? make_float2(-INFINITY, __int_as_float(0x7fffffff))
-                              : make_float2(-INFINITY, 0.f));
-          if (a.greedy) {
-            float av;
-            int32_t ai;
-            group_amax(reg, av, ai);
-            if (grp_sub == 0 && row_on) ctl->tok[n] = ai;
-            if (a.mode == MODE_CYCLE) {
-              const bool al = row_on && ctl->alive[n];
-              load_slice(a.tpart + (((int64_t)par * (K + 1) + i) * N + n) * kMaxG, al, reg,
-                         make_float2(-INFINITY, __int_as_float(0x7fffffff)));
-              float tv;
-              int32_t tam;
-              group_amax(reg, tv, tam);
-              if (grp_sub == 0 && al) {
-                const int b = g * N + n;
-                const bool acc = tam == ai;
-                if (cta == 0) a.out[(int64_t)b * (K + 1) + i] = acc ? ai : tam;
-                if (!acc) {
+          grid_arrive();
+          mark(g, i, 3);
+          // background while the barrier completes: next target row, rows alive so far
+          if (attempt == 0 && a.mode == MODE_CYCLE) target_row_stats(g, par, i + 1, nb_g);
+          mark(g, i, 4);
+          if (!grid_wait()) {
+            failed = true;
+            break;
+          }
+          mark(g, i, 5);
+          // ---------------- row reducers publish one record per row
+          if (tid == 0) {
+            ctl->n_owned = 0;
+            ctl->redo = 0;
+          }
+          const int mine = reduce_rows(0, g, par, i, nb_g, fast);
+          mark(g, i, 12);
+          if (!records_hop(mine, nb_g)) {
+            failed = true;
+            break;
+          }
+          for (int n = tid; n < nb_g; n += kComputeThreads) {
+            const Rec r = load_rec(a.rec + ((int64_t)par * (K + 2) + i) * N + n);
+            const int b = g * N + n;
+            if (a.greedy) {
+              ctl->tok[n] = r.token;
+              if (cta == 0 && a.draft) a.draft[(int64_t)b * K + i] = r.token;
+              if (a.mode == MODE_CYCLE && ctl->alive[n]) {
+                if (cta == 0) a.out[(int64_t)b * (K + 1) + i] = r.acc ? r.token : r.tam;
+                if (!r.acc) {
                   ctl->alive[n] = 0;
                   ctl->stoprow[n] = i;
                 }
               }
-            }
-          } else {
-            float M, S;
-            group_ms(reg, M, S);
-            mark(g, i, 12);
-            const int b = g * N + n;
-            const float u = philox_uniform(a.seed, a.cycle, (uint32_t)b, (uint32_t)i, TAG_DRAFT);
-            const float tgt = u * S;
-            int own;
-            float before;
-            bool fb;
-            const bool holder = group_owner(reg, 0, M, tgt, own, before, fb);
-            mark(g, i, 13);
-            if (row_on) {
-              if (grp_sub == 0) {
-                ctl->M[n] = M;
-                ctl->S[n] = S;
-              }
-              if (holder && own == cta) {
+            } else {
+              ctl->M[n] = r.M;
+              ctl->S[n] = r.S;
+              ctl->ref[n] = r.Mx;
+              ctl->Mt[n] = r.Mt;
+              ctl->St[n] = r.St;
+              if (r.flags & 1) ctl->redo = 1;
+              if (r.owner == cta) {
                 const int slot = atomicAdd(&ctl->n_owned, 1);
                 ctl->owned[slot] = n;
-                ctl->obtarget[slot] = fb ? INFINITY : tgt - before;
+                ctl->obtarget[slot] = r.trem;
               }
-            }
-            if (a.mode == MODE_CYCLE) {
-              // target statistics of row i for the rows still alive (used by owners)
-              const bool al = row_on && ctl->alive[n];
-              load_slice(a.tpart + (((int64_t)par * (K + 1) + i) * N + n) * kMaxG, al, reg,
-                         make_float2(-INFINITY, 0.f));
-              float Mt, St;
-              group_ms(reg, Mt, St);
-              if (grp_sub == 0 && al) {
-                ctl->Mt[n] = Mt;
-                ctl->St[n] = St;
-              }
-              mark(g, i, 14);
             }
           }
+          named_sync();
+          mark(g, i, 6);
+          if (!ctl->redo) break;  // read after the barrier: the same in every thread
+          fast = false;           // exact statistics, re-read from tensor memory
         }
-        named_sync();
-        mark(g, i, 6);
+        if (failed) break;
 
         if (a.greedy) {
-          if (cta == 0)
-            for (int n = tid; n < nb_g; n += kComputeThreads)
-              if (a.draft) a.draft[(int64_t)(g * N + n) * K + i] = ctl->tok[n];
           tc_fence_before();
           named_sync();
           if (TC && tid == 0) mbar_arrive(&ctl->tfree);
@@ -1015,43 +1191,37 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           // ---------------- owners: bucket walk, then batched bucket scans
           walk_and_assign(false);
           mark(g, i, 15);
-          const int cnt = ctl->wcount[warp];
-          for (int bs = 0; bs < cnt; bs += kOwnBatch) {
+          const int n_owned = ctl->n_owned;
+          if (warp < n_owned) {  // owned rows o = warp, warp + 8, ... (n_owned <= N <= 64)
             int oo[kOwnBatch];
             float dv[kOwnBatch], td[kOwnBatch], zd[kOwnBatch], qd[kOwnBatch];
             int dtok[kOwnBatch];
 #pragma unroll
             for (int j = 0; j < kOwnBatch; ++j) {
-              oo[j] = bs + j < cnt ? ctl->wlist[warp][bs + j] : -1;
+              oo[j] = warp + 8 * j < n_owned ? warp + 8 * j : -1;
               dtok[j] = 0;
+              dv[j] = oo[j] < 0 ? 0.f : zbuf[oo[j] * 32 + lane];
             }
 #pragma unroll
             for (int j = 0; j < kOwnBatch; ++j) {
-              dv[j] = 0.f;
               if (oo[j] < 0) continue;
-              const int cl = ctl->obucket[oo[j]] >> 2, n = ctl->owned[oo[j]];
-              tmem_ld1(taddr + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(cl * N + n), &dv[j]);
-            }
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < kOwnBatch; ++j) {
-              if (oo[j] < 0) continue;
-              const int cl = ctl->obucket[oo[j]] >> 2, n = ctl->owned[oo[j]];
+              const int bk = ctl->obucket[oo[j]], n = ctl->owned[oo[j]];
+              const int v0 = (chunk0 + (bk >> 2)) * kCH + (bk & 3) * 32;  // bucket's first token
               const float M = ctl->M[n], S = ctl->S[n];
-              const int v = (chunk0 + cl) * kCH + q4 * 32 + lane;
+              const int v = v0 + lane;
               const bool valid = v < V;
               const float z = valid ? dv[j] : -INFINITY;  // z = base + bias, kept in tensor memory
               const float e = valid ? exp2f((z - M) * k) : 0.f;
               const int wl = bucket_scan(e, ctl->obtarget[oo[j]]);
-              dtok[j] = (chunk0 + cl) * kCH + q4 * 32 + wl;
+              dtok[j] = v0 + wl;
               zd[j] = __shfl_sync(FULL, z, wl);
               qd[j] = exp2f((zd[j] - M) * k) / S;
             }
             const bool cyc = a.mode == MODE_CYCLE;
 #pragma unroll
             for (int j = 0; j < kOwnBatch; ++j) {
-              const int oj = oo[j] < 0 ? 0 : oo[j];
-              const int n = min(ctl->owned[oj], nb_g - 1);
+              const int oj = oo[j] < 0 ? warp : oo[j];  // slot "warp" is owned
+              const int n = ctl->owned[oj];
               const int dt = oo[j] < 0 ? 0 : min(max(dtok[j], 0), V - 1);
               td[j] = cyc ? ld_elem(target, ((int64_t)(g * N + n) * (K + 1) + i) * V + dt) : 0.f;
             }
@@ -1068,7 +1238,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
                 const float Mt = ctl->Mt[n], St = ctl->St[n];
                 pd = exp2f((td[j] - Mt) * k) / St;
                 const float ratio = exp2f(((td[j] - Mt) - (zd[j] - M)) * k) * (S / St);
-                const float uacc = philox_uniform(a.seed, a.cycle, (uint32_t)b, (uint32_t)i, TAG_ACCEPT);
+                const float uacc = philox_uniform(a.seed, a.cycle, a.row0 + (uint32_t)b, (uint32_t)i, TAG_ACCEPT);
                 accept = uacc < fminf(ratio, 1.0f) ? 1 : 0;
               }
               if (lane == 0) {
@@ -1078,10 +1248,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
                 if (a.q_draft) a.q_draft[(int64_t)b * K + i] = qd[j];
                 if (alive) {
                   if (a.p_draft) a.p_draft[(int64_t)b * K + i] = pd;
-                  if (accept)
-                    a.out[(int64_t)b * (K + 1) + i] = dtok[j];
-                  else
-                    a.stopinfo[(int64_t)par * N + n] = StopInfo{i, ctl->Mt[n], ctl->St[n], M, S};
+                  if (accept) a.out[(int64_t)b * (K + 1) + i] = dtok[j];
                 }
               }
             }
@@ -1115,10 +1282,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               prefetch_l2_bulk(base + ((int64_t)(g * N + n) * K + i) * V + vslice_lo, sl);
               ctl->alive[n] = 0;
               ctl->stoprow[n] = i;
-              ctl->zM[n] = ctl->M[n];
+              ctl->zM[n] = ctl->M[n];  // draft statistics of the stop row
               ctl->zS[n] = ctl->S[n];
-              ctl->Mt[n] = __ldcg(&a.stopinfo[(int64_t)par * N + n].mt);
-              ctl->St[n] = __ldcg(&a.stopinfo[(int64_t)par * N + n].st);
+              ctl->fMt[n] = ctl->Mt[n];  // target statistics of the stop row
+              ctl->fSt[n] = ctl->St[n];
             }
           }
           named_sync();
@@ -1140,28 +1307,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
         }
         mark(g, K, 1);
         {
-          // target statistics of row K for the rows that accepted every draft
-          const int n = grp_n;
-          const bool al = n < nb_g && ctl->alive[n];
-          float2 reg[MAXC];
-          load_slice(a.tpart + (((int64_t)par * (K + 1) + K) * N + n) * kMaxG, al, reg,
-                     a.greedy ? make_float2(-INFINITY, __int_as_float(0x7fffffff))
-                              : make_float2(-INFINITY, 0.f));
-          if (a.greedy) {
-            float tv;
-            int32_t tam;
-            group_amax(reg, tv, tam);
-            if (grp_sub == 0 && al && cta == 0) a.out[(int64_t)(g * N + n) * (K + 1) + K] = tam;
-          } else {
-            float Mt, St;
-            group_ms(reg, Mt, St);
-            if (grp_sub == 0 && al) {
-              ctl->Mt[n] = Mt;
-              ctl->St[n] = St;
+          const int mine = reduce_rows(1, g, par, K, nb_g, false);
+          if (!records_hop(mine, nb_g)) {
+            failed = true;
+            break;
+          }
+          for (int n = tid; n < nb_g; n += kComputeThreads) {
+            if (!ctl->alive[n]) continue;
+            const Rec r = load_rec(a.rec + ((int64_t)par * (K + 2) + K) * N + n);
+            if (a.greedy) {
+              if (cta == 0) a.out[(int64_t)(g * N + n) * (K + 1) + K] = r.tam;
+            } else {
+              ctl->fMt[n] = r.Mt;
+              ctl->fSt[n] = r.St;
             }
           }
+          named_sync();
         }
-        named_sync();
         if (!a.greedy) {
           // ---------------- final step: residual at the stop row, or the bonus
           for (int n = tid; n < N; n += kComputeThreads) {
@@ -1198,7 +1360,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               const int n = n0 + j;
               float r = 0.f, p = 0.f;
               if (valid && n < nb_g) {
-                p = exp2f((tv[j] - ctl->Mt[n]) * k) / ctl->St[n];
+                p = exp2f((tv[j] - ctl->fMt[n]) * k) / ctl->fSt[n];
                 r = p;
                 if (!ctl->alive[n])
                   r = fmaxf(p - exp2f((d[j] + bvv[j] - ctl->zM[n]) * k) / ctl->zS[n], 0.f);
@@ -1225,7 +1387,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               P += __shfl_xor_sync(FULL, P, off);
             }
             if (grp_sub == 0)
-              a.dpart[(((int64_t)par * (K + 1) + K) * N + n) * kMaxG + cta] = make_float2(R, P);
+              a.dpart[(((int64_t)par * (K + 1) + K) * N + n) * kMaxG + cta] = make_float4(R, P, 0.f, 0.f);
           }
           mark(g, K, 3);
           if (!grid_barrier()) {
@@ -1234,87 +1396,60 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           }
           mark(g, K, 4);
           if (tid == 0) ctl->n_owned = 0;
-          named_sync();
-          {
-            const int n = grp_n;
-            const bool row_on = n < nb_g;
-            float2 reg[MAXC];
-            load_slice(a.dpart + (((int64_t)par * (K + 1) + K) * N + n) * kMaxG, row_on, reg,
-                       make_float2(0.f, 0.f));
-            float lr = 0.f, lp = 0.f;
-#pragma unroll
-            for (int j = 0; j < MAXC; ++j) {
-              lr += reg[j].x;
-              lp += reg[j].y;
-            }
-            float Rt = lr, Pt = lp;
-#pragma unroll
-            for (int off = TPB / 2; off >= 1; off >>= 1) {
-              Rt += __shfl_xor_sync(FULL, Rt, off);
-              Pt += __shfl_xor_sync(FULL, Pt, off);
-            }
-            const bool use_p = !(Rt > 0.f);
-            const int b = g * N + n;
-            const int row = (row_on && ctl->alive[n]) ? K : (row_on ? ctl->stoprow[n] : 0);
-            const float u = philox_uniform(a.seed, a.cycle, (uint32_t)b, (uint32_t)row, TAG_RESAMPLE);
-            const float tgt = u * (use_p ? Pt : Rt);
-            int own;
-            float before;
-            bool fb;
-            const bool holder = group_owner(reg, use_p ? 2 : 1, 0.f, tgt, own, before, fb);
-            if (row_on) {
-              if (grp_sub == 0) ctl->S[n] = use_p ? 1.f : 0.f;  // which mass the scan uses
-              if (holder && own == cta) {
-                const int slot = atomicAdd(&ctl->n_owned, 1);
-                ctl->owned[slot] = n;
-                ctl->obtarget[slot] = fb ? INFINITY : tgt - before;
-              }
+          const int mine = reduce_rows(2, g, par, K, nb_g, false);
+          if (!records_hop(mine, nb_g)) {
+            failed = true;
+            break;
+          }
+          for (int n = tid; n < nb_g; n += kComputeThreads) {
+            const Rec r = load_rec(a.rec + ((int64_t)par * (K + 2) + K + 1) * N + n);
+            ctl->S[n] = (r.flags & 2) ? 1.f : 0.f;  // which mass the scan uses
+            if (r.owner == cta) {
+              const int slot = atomicAdd(&ctl->n_owned, 1);
+              ctl->owned[slot] = n;
+              ctl->obtarget[slot] = r.trem;
             }
           }
           named_sync();
           walk_and_assign(true);
-          const int cnt = ctl->wcount[warp];
-          for (int bs = 0; bs < cnt; bs += kOwnBatch) {
+          const int n_owned = ctl->n_owned;
+          if (warp < n_owned) {  // owned rows o = warp, warp + 8, ...
             int oo[kOwnBatch];
             float dv[kOwnBatch], tvv[kOwnBatch], bvv[kOwnBatch];
 #pragma unroll
-            for (int j = 0; j < kOwnBatch; ++j) oo[j] = bs + j < cnt ? ctl->wlist[warp][bs + j] : -1;
-#pragma unroll
             for (int j = 0; j < kOwnBatch; ++j) {
-              dv[j] = 0.f;
-              if (oo[j] < 0) continue;
-              const int cl = ctl->obucket[oo[j]] >> 2, n = ctl->owned[oo[j]];
-              tmem_ld1(taddr + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(cl * N + n), &dv[j]);
+              oo[j] = warp + 8 * j < n_owned ? warp + 8 * j : -1;
+              dv[j] = oo[j] < 0 ? 0.f : zbuf[oo[j] * 32 + lane];
             }
-            tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < kOwnBatch; ++j) {  // loads from clamped valid addresses
-              const int oj = oo[j] < 0 ? 0 : oo[j];
-              const int cl = ctl->obucket[oj] >> 2, n = min(ctl->owned[oj], nb_g - 1);
+              const int oj = oo[j] < 0 ? warp : oo[j];  // slot "warp" is owned
+              const int bk = ctl->obucket[oj], n = ctl->owned[oj];
               const int b = g * N + n;
               const int row = ctl->alive[n] ? K : ctl->stoprow[n];
-              const int v = min((chunk0 + cl) * kCH + q4 * 32 + lane, V - 1);
+              const int v = min((chunk0 + (bk >> 2)) * kCH + (bk & 3) * 32 + lane, V - 1);
               tvv[j] = ld_elem(target, ((int64_t)b * (K + 1) + row) * V + v);
               bvv[j] = ld_elem(base, ((int64_t)b * K + min(row, K - 1)) * V + v);
             }
 #pragma unroll
             for (int j = 0; j < kOwnBatch; ++j) {
               if (oo[j] < 0) continue;
-              const int cl = ctl->obucket[oo[j]] >> 2, n = ctl->owned[oo[j]];
+              const int bk = ctl->obucket[oo[j]], n = ctl->owned[oo[j]];
+              const int v0 = (chunk0 + (bk >> 2)) * kCH + (bk & 3) * 32;
               const int b = g * N + n;
               const bool use_p = ctl->S[n] != 0.f;
               const bool bonus = ctl->alive[n] != 0;
               const int row = bonus ? K : ctl->stoprow[n];
-              const int v = (chunk0 + cl) * kCH + q4 * 32 + lane;
+              const int v = v0 + lane;
               float w = 0.f;
               if (v < V) {
-                const float p = exp2f((tvv[j] - ctl->Mt[n]) * k) / ctl->St[n];
+                const float p = exp2f((tvv[j] - ctl->fMt[n]) * k) / ctl->fSt[n];
                 w = p;
                 if (!bonus && !use_p)
                   w = fmaxf(p - exp2f((dv[j] + bvv[j] - ctl->zM[n]) * k) / ctl->zS[n], 0.f);
               }
               const int wl = bucket_scan(w, ctl->obtarget[oo[j]]);
-              if (lane == 0) a.out[(int64_t)b * (K + 1) + row] = (chunk0 + cl) * kCH + q4 * 32 + wl;
+              if (lane == 0) a.out[(int64_t)b * (K + 1) + row] = v0 + wl;
             }
           }
           mark(g, K, 5);
@@ -1356,6 +1491,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
       __threadfence();
       hdr->bar = 0;
       hdr->tok = 0;
+      hdr->rec = 0;
       hdr->abort = 0;
       __threadfence();
       atomicExch(&hdr->exit_count, 0u);
@@ -1371,7 +1507,7 @@ size_t smem_bytes(int r, int nc) {
   const size_t u = TC ? (size_t)nkb * N * 128 : (size_t)N * r * 4;
   s += (u + 1023) & ~size_t(1023);
   s += (size_t)kNBS * N * kCH * sizeof(T);
-  s += (size_t)nc * 4 * N * sizeof(float2);
+  s += bucket_region_bytes(nc, N);
   s += sizeof(Ctl<N>);
   return s;
 }
@@ -1441,13 +1577,17 @@ namespace {
 size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 }  // namespace
 
-// Workspace body: trace | dpart | tpart | tokens | accf | stopinfo, each 256-byte aligned.
+// Workspace body: trace | dpart | tpart | tokens | accf | records, each 256-byte aligned.
 size_t cycle_trace_bytes(int K) { return a256(sizeof(uint64_t) * (size_t)(K + 2) * kTracePhases); }
+namespace {
+size_t dpart_bytes(int K, int N) { return a256(sizeof(float4) * 2 * (size_t)(K + 1) * N * kMaxG); }
+size_t tpart_bytes(int K, int N) { return a256(sizeof(float2) * 2 * (size_t)(K + 1) * N * kMaxG); }
+size_t tok_bytes(int K, int N) { return a256(sizeof(int32_t) * 2 * (size_t)K * N); }
+size_t rec_bytes(int K, int N) { return a256(sizeof(Rec) * 2 * (size_t)(K + 2) * N); }
+}  // namespace
 size_t cycle_ws_bytes(int K, const CycleGeom& g) {
-  const size_t part = sizeof(float2) * 2 * (size_t)(K + 1) * g.N * kMaxG;
-  const size_t tok = sizeof(int32_t) * 2 * (size_t)K * g.N;
-  return cycle_trace_bytes(K) + 2 * a256(part) + 2 * a256(tok) +
-         a256(sizeof(StopInfo) * 2 * g.N);
+  return cycle_trace_bytes(K) + dpart_bytes(K, g.N) + tpart_bytes(K, g.N) + 2 * tok_bytes(K, g.N) +
+         rec_bytes(K, g.N);
 }
 
 cudaError_t launch_cycle(const CycleLaunch& L, const CycleGeom& g, WsHeader* hdr, uint8_t* body,
@@ -1468,15 +1608,17 @@ cudaError_t launch_cycle(const CycleLaunch& L, const CycleGeom& g, WsHeader* hdr
   a.q_draft = L.q_draft;
   a.biased_out = L.biased_out;
   a.hdr = hdr;
-  const size_t part = a256(sizeof(float2) * 2 * (size_t)(L.K + 1) * g.N * kMaxG);
-  const size_t tok = a256(sizeof(int32_t) * 2 * (size_t)L.K * g.N);
   a.trace = L.trace ? reinterpret_cast<uint64_t*>(body) : nullptr;
   body += cycle_trace_bytes(L.K);
-  a.dpart = reinterpret_cast<float2*>(body);
-  a.tpart = reinterpret_cast<float2*>(body + part);
-  a.tokens = reinterpret_cast<int32_t*>(body + 2 * part);
-  a.accf = reinterpret_cast<int32_t*>(body + 2 * part + tok);
-  a.stopinfo = reinterpret_cast<StopInfo*>(body + 2 * part + 2 * tok);
+  a.dpart = reinterpret_cast<float4*>(body);
+  body += dpart_bytes(L.K, g.N);
+  a.tpart = reinterpret_cast<float2*>(body);
+  body += tpart_bytes(L.K, g.N);
+  a.tokens = reinterpret_cast<int32_t*>(body);
+  body += tok_bytes(L.K, g.N);
+  a.accf = reinterpret_cast<int32_t*>(body);
+  body += tok_bytes(L.K, g.N);
+  a.rec = reinterpret_cast<Rec*>(body);
   a.B = L.B;
   a.K = L.K;
   a.V = L.V;
@@ -1489,6 +1631,7 @@ cudaError_t launch_cycle(const CycleLaunch& L, const CycleGeom& g, WsHeader* hdr
   a.ngroups = (L.B + g.N - 1) / g.N;
   a.k = L.greedy ? 1.0f : 1.4426950408889634f / L.temperature;
   a.seed = L.seed;
+  a.row0 = L.row0;
   a.cycle = L.cycle;
   a.spin = L.spin;
   if (L.dtype == SPEC_BF16) {

@@ -36,7 +36,7 @@ template <typename T, typename TD>
 cudaError_t launch_verify(const T* target, const TD* draft_logits, const int32_t* draft,
                           int32_t* out, int32_t* tau, float* p_draft, float* q_draft, int B,
                           int K, int V, float temperature, int greedy, uint64_t seed,
-                          uint64_t cycle, uint8_t* ws_body, WsHeader* hdr, int num_sms,
+                          uint64_t cycle, uint32_t row0, uint8_t* ws_body, WsHeader* hdr, int num_sms,
                           cudaStream_t st, int* launches);
 
 // ---- Fused persistent draft (+ verify) ---------------------------------------
@@ -73,6 +73,7 @@ struct CycleLaunch {
   int B, K, V, r, dtype, mode, greedy;
   float temperature;
   uint64_t seed, cycle, spin;
+  uint32_t row0;  // global index of batch row 0 (Philox counter word 1)
   bool trace;
 };
 

@@ -148,7 +148,7 @@ template <typename T, typename TD>
 __global__ void k_accept(const T* __restrict__ target, const TD* __restrict__ draft_logits,
                          const int32_t* __restrict__ draft, const RowPartial* __restrict__ tstats,
                          const RowPartial* __restrict__ dstats, int B, int K, int V, int nseg,
-                         float k, int greedy, uint64_t seed, uint64_t cycle,
+                         float k, int greedy, uint64_t seed, uint64_t cycle, uint32_t row0,
                          int32_t* __restrict__ out, int32_t* __restrict__ tau,
                          float* __restrict__ p_draft, float* __restrict__ q_draft,
                          StopInfo* __restrict__ stop, WsHeader* hdr) {
@@ -187,7 +187,7 @@ __global__ void k_accept(const T* __restrict__ target, const TD* __restrict__ dr
     // ratio p/q from one exponent of small magnitude
     float a = exp2f(((td - tp.m) - (zd - dp.m)) * k) * (dp.s / tp.s);
     a = fminf(a, 1.0f);
-    const float u = philox_uniform(seed, cycle, (uint32_t)b, (uint32_t)i, TAG_ACCEPT);
+    const float u = philox_uniform(seed, cycle, row0 + (uint32_t)b, (uint32_t)i, TAG_ACCEPT);
     if (u < a) {
       out[(int64_t)b * (K + 1) + i] = d;
       continue;
@@ -259,7 +259,8 @@ template <typename T, typename TD>
 __global__ void __launch_bounds__(kThreads) k_residual_pick(
     const T* __restrict__ target, const TD* __restrict__ draft_logits,
     const StopInfo* __restrict__ stop, const float2* __restrict__ part, int B, int K, int V,
-    int seg_len, int nseg, float k, uint64_t seed, uint64_t cycle, int32_t* __restrict__ out) {
+    int seg_len, int nseg, float k, uint64_t seed, uint64_t cycle, uint32_t row0,
+    int32_t* __restrict__ out) {
   __shared__ float sh_target;
   __shared__ int sh_seg, sh_use_p;
   __shared__ float wsum[kThreads / 32];
@@ -276,7 +277,7 @@ __global__ void __launch_bounds__(kThreads) k_residual_pick(
     }
     const int use_p = !(R > 0.f);
     const float tot = use_p ? P : R;
-    const float u = philox_uniform(seed, cycle, (uint32_t)b, (uint32_t)si.j, TAG_RESAMPLE);
+    const float u = philox_uniform(seed, cycle, row0 + (uint32_t)b, (uint32_t)si.j, TAG_RESAMPLE);
     const float tgt = u * tot;
     float c = 0.f;
     int seg = -1, lastpos = 0;
@@ -368,7 +369,8 @@ template <typename T, typename TD>
 cudaError_t launch_verify(const T* target, const TD* draft_logits, const int32_t* draft,
                           int32_t* out, int32_t* tau, float* p_draft, float* q_draft, int B,
                           int K, int V, float temperature, int greedy, uint64_t seed,
-                          uint64_t cycle, uint8_t* ws_body, WsHeader* hdr, int num_sms,
+                          uint64_t cycle, uint32_t row0, uint8_t* ws_body, WsHeader* hdr,
+                          int num_sms,
                           cudaStream_t st, int* launches) {
   const int seg_len = verify_seg_len(V);
   const int nseg = (V + seg_len - 1) / seg_len;
@@ -394,14 +396,14 @@ cudaError_t launch_verify(const T* target, const TD* draft_logits, const int32_t
     ++*launches;
   }
   k_accept<T, TD><<<(B + 127) / 128, 128, 0, st>>>(target, draft_logits, draft, tstats, dstats, B,
-                                                   K, V, nseg, k, greedy, seed, cycle, out, tau,
+                                                   K, V, nseg, k, greedy, seed, cycle, row0, out, tau,
                                                    p_draft, q_draft, stop, hdr);
   ++*launches;
   if (!greedy) {
     k_residual_part<T, TD><<<grid_for((int64_t)B * nseg), kThreads, 0, st>>>(
         target, draft_logits, stop, B, K, V, seg_len, nseg, k, part);
     k_residual_pick<T, TD><<<B, kThreads, 0, st>>>(target, draft_logits, stop, part, B, K, V,
-                                                   seg_len, nseg, k, seed, cycle, out);
+                                                   seg_len, nseg, k, seed, cycle, row0, out);
     *launches += 2;
   }
   return cudaGetLastError();
@@ -419,8 +421,8 @@ size_t verify_ws_bytes(int B, int K, int V) {
 #define INST(T, TD)                                                                           \
   template cudaError_t launch_verify<T, TD>(const T*, const TD*, const int32_t*, int32_t*,    \
                                             int32_t*, float*, float*, int, int, int, float,   \
-                                            int, uint64_t, uint64_t, uint8_t*, WsHeader*, int, \
-                                            cudaStream_t, int*);
+                                            int, uint64_t, uint64_t, uint32_t, uint8_t*,      \
+                                            WsHeader*, int, cudaStream_t, int*);
 INST(float, float)
 INST(__nv_bfloat16, __nv_bfloat16)
 INST(__nv_bfloat16, float)

@@ -99,7 +99,10 @@ typedef struct {
   uint64_t cycle;        /* Philox counter words 2..3 (advance it every cycle) */
   uint64_t spin_limit;   /* polls before a device wait gives up; 0 = default (about 2 s) */
   uint32_t flags;        /* SPEC_FLAG_* */
-  uint32_t reserved;
+  uint32_t row_offset;   /* global index of batch row 0: row b draws from Philox counter word
+                            row_offset + b, so a batch split into shards (calls or GPUs) with
+                            their starting rows draws exactly what one call over it draws;
+                            row_offset + B must not exceed 2^31 */
 } spec_params;
 
 /* Bytes of device workspace the calls need for these parameters on the

@@ -48,6 +48,7 @@ def _p(**kw):
     (dict(r=300), sd.SPEC_ERR_INVALID_ARG),
     (dict(temperature=0.0), sd.SPEC_ERR_INVALID_ARG),
     (dict(V=1001), sd.SPEC_ERR_UNSUPPORTED),
+    (dict(row_offset=2**31 - 3), sd.SPEC_ERR_INVALID_ARG),  # row_offset + B beyond 2^31
 ])
 def test_host_validation_before_launch(kw, code):
     L = sd.lib()
@@ -76,3 +77,39 @@ def test_greedy_allows_zero_temperature_shape_check():
     # passes the temperature rule, then fails on the vocabulary alignment rule
     assert L.spec_cycle(ctypes.byref(p), *([fake] * 6), fake, fake, None, None, fake,
                         None) == sd.SPEC_ERR_UNSUPPORTED
+
+
+def test_params_struct_matches_header():
+    """The ctypes mirror lists spec_params' fields in the header's order, with
+    the header's integer widths, so the binding and the library agree on
+    every offset."""
+    text = open(os.path.join(ROOT, "include", "specdec.h")).read()
+    body = re.search(r"typedef struct \{(.*?)\} spec_params;", text, flags=re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = re.findall(r"\b(u?int\d+_t|float)\s+(\w+)\s*;", body)
+    ctype = {"int32_t": ctypes.c_int32, "uint32_t": ctypes.c_uint32, "uint64_t": ctypes.c_uint64,
+             "float": ctypes.c_float}
+    assert [(n, ctype[t]) for t, n in fields] == list(sd.SpecParams._fields_)
+
+
+def test_params_offsets_match_the_c_compiler(tmp_path):
+    """Field offsets and size of spec_params as the host C compiler lays them
+    out, against the ctypes mirror."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no host C compiler")
+    names = [n for n, _ in sd.SpecParams._fields_]
+    src = tmp_path / "probe.c"
+    lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "specdec.h"', "int main(void) {",
+             '  printf("%zu\\n", sizeof(spec_params));']
+    lines += [f'  printf("%zu\\n", offsetof(spec_params, {n}));' for n in names]
+    lines += ["  return 0;", "}"]
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "probe"
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], check=True, capture_output=True,
+                                          text=True).stdout.split()]
+    want = [ctypes.sizeof(sd.SpecParams)] + [getattr(sd.SpecParams, n).offset for n in names]
+    assert got == want

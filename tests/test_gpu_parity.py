@@ -36,10 +36,11 @@ def _np(t):
     return t.cpu().numpy()
 
 
-def gpu_cycle(w, d, greedy=False, T=None, seed=0, cyc=0, flags=0, spin=0, dd=None):
+def gpu_cycle(w, d, greedy=False, T=None, seed=0, cyc=0, flags=0, spin=0, dd=None, row_offset=0):
     T = w.temperature if T is None else T
     p = sd.Params(B=d["base"].shape[0], K=w.K, V=w.V, r=w.r, dtype=w.dtype, temperature=T,
-                  greedy=greedy, seed=seed, cycle=cyc, flags=flags, spin_limit=spin)
+                  greedy=greedy, seed=seed, cycle=cyc, flags=flags, spin_limit=spin,
+                  row_offset=row_offset)
     dd = dd or _dev(d)
     ws = sd.make_workspace(p)
     o = sd.alloc_outputs(p)
@@ -211,6 +212,54 @@ def test_cycle_vs_oracle(name, w, greedy, T):
         total_flag += compare_cycle(g, o, w.K)
         check_invariants(g["out"], g["tau"], g["draft"], w.K)
     assert total_flag <= max(1, d["base"].shape[0] // 10)
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_cycle_sharded_blocks_match_the_whole_batch(world):
+    """Row blocks run as separate calls, each with its first global row as
+    row_offset (what every rank of a batch-sharded job does), give the oracle's
+    output for those rows of the whole batch."""
+    from draft_sampling_verification_head_b200 import shard
+    w = CASES[2][1]  # B=70: blocks of 35 / 24,23,23 rows, one and two row groups
+    d = synth.make(w)
+    o = orc_cycle(w, d, T=0.8, seed=21, cyc=4)
+    total_flag = 0
+    got = {k: [] for k in ("draft", "out", "tau", "p_draft", "q_draft")}
+    for r in range(world):
+        b0, b1 = shard.shard_range(w.B, world, r)
+        blk = {k: (v if k in ("U", "W") else v[b0:b1].contiguous()) for k, v in d.items()}
+        g = gpu_cycle(w, blk, T=0.8, seed=21, cyc=4, row_offset=b0)
+        for k in got:
+            got[k].append(g[k])
+    g = {k: np.concatenate(v) for k, v in got.items()}
+    total_flag += compare_cycle(g, o, w.K)
+    check_invariants(g["out"], g["tau"], g["draft"], w.K)
+    assert total_flag <= max(1, w.B // 10)
+
+
+def test_verify_block_row_offset():
+    B, K, V = 9, 4, 3000
+    w = synth.Workload("vo", B=B, K=K, V=V, r=8, dtype="bf16", sigma=0.7, seed=52)
+    d = synth.make(w)
+    P = oracle.Params(B=B, K=K, V=V, r=0, dtype="bf16", temperature=1.0, seed=4, cycle=1)
+    drafts = oracle.draft(P, synth.to_numpy_raw(d["base"]), np.zeros((V, 0), np.uint16),
+                          np.zeros((0, V), np.uint16), d["last_token"].numpy())["draft"]
+    o = oracle.verify(P, synth.to_numpy_raw(d["target"]), synth.to_numpy_raw(d["base"]), drafts)
+    b0 = 5  # the block of rows 5..8, called on its own
+    p = sd.Params(B=B - b0, K=K, V=V, r=0, dtype="bf16", temperature=1.0, seed=4, cycle=1,
+                  row_offset=b0)
+    ws = sd.make_workspace(p)
+    outs = sd.alloc_outputs(p)
+    sd.verify_block(p, d["target"][b0:].contiguous().cuda(), d["base"][b0:].contiguous().cuda(),
+                    torch.from_numpy(drafts[b0:].copy()).cuda(), outs["out"], outs["tau"],
+                    outs["p_draft"], outs["q_draft"], ws)
+    assert sd.sync_status(ws) == sd.SPEC_OK
+    gpu = {k: _np(v) for k, v in outs.items()}
+    gpu["draft"] = drafts[b0:]
+    ref = {k: (v[b0:] if isinstance(v, np.ndarray) else v) for k, v in o.items()}
+    ref["draft"] = drafts[b0:]
+    ref["flag_draft"] = np.full(B - b0, K, np.int32)
+    compare_cycle(gpu, ref, K)
 
 
 def test_cycle_deterministic():

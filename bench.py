@@ -57,12 +57,15 @@ def early_exit_bytes(w, tau) -> float:
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms from before
+    the warm-up to after the timed region; the summary keeps the samples read
+    between mark_start() and mark_end() (host clock)."""
 
     def __init__(self, gpu_index: int):
         self.idx = gpu_index
-        self.samples = []
+        self.samples = []  # (host time, fields)
         self.proc = None
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -81,7 +84,13 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.samples.append([x.strip() for x in line.split(",")])
+            self.samples.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -92,16 +101,19 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(s[1]) for s in self.samples if len(s) > 8 and s[1].replace(".", "").isdigit()]
-        mx = [float(s[2]) for s in self.samples if len(s) > 8 and s[2].replace(".", "").isdigit()]
+        rows = [f for t, f in self.samples if len(f) > 8 and self.t0 is not None and
+                self.t1 is not None and self.t0 <= t <= self.t1]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        num = lambda x: x.replace(".", "", 1).isdigit()
+        sm = [float(f[1]) for f in rows if num(f[1])]
+        mx = [float(f[2]) for f in rows if num(f[2])]
+        pw = [float(f[3]) for f in rows if num(f[3])]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[j] for s in self.samples if len(s) > 8
-                          for j in range(4) if s[5 + j].lower() == "active"})
+        reasons = sorted({names[j] for f in rows for j in range(4) if f[5 + j].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(self.samples)}
+                "power_w": statistics.median(pw) if pw else None, "samples": len(rows)}
 
 
 def measured_peak():
@@ -199,19 +211,19 @@ def run_ours(args, rank, world, local_rank):
     import synth
     import draft_sampling_verification_head_b200 as sd
 
+    from draft_sampling_verification_head_b200 import shard
+
     torch.cuda.set_device(local_rank)
-    dist = None
-    if world > 1:
-        import torch.distributed as dist_mod
-        import datetime
-        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-        dist = dist_mod
+    multi = shard.init("nccl", timeout_s=120)
     w = synth.WORKLOADS[WORKLOAD]
-    d = synth.make(w, seed=w.seed + 1000 * rank)  # each rank its own batch of B rows
+    # Weak scaling: the job's batch is world x B rows; rank r holds rows
+    # [r*B, (r+1)*B) (its own seeded logits) and draws with row_offset r*B.
+    row0, row1 = shard.shard_range(w.B * world, world, rank)
+    d = synth.make(w, seed=w.seed + 1000 * rank)
     dev = torch.device("cuda", local_rank)
     dd = {k: v.to(dev) for k, v in d.items()}
-    p = sd.Params(B=w.B, K=w.K, V=w.V, r=w.r, dtype=w.dtype, temperature=w.temperature,
-                  seed=w.seed + rank, cycle=0)
+    p = sd.Params(B=row1 - row0, K=w.K, V=w.V, r=w.r, dtype=w.dtype, temperature=w.temperature,
+                  seed=w.seed, cycle=0, row_offset=row0)
     ws = sd.make_workspace(p)
     o = sd.alloc_outputs(p)
     stream = torch.cuda.current_stream()
@@ -221,38 +233,34 @@ def run_ours(args, rank, world, local_rank):
         sd.cycle(p, dd["base"], dd["target"], dd["U"], dd["W"], dd["last_token"], o["draft"],
                  o["out"], o["tau"], o["p_draft"], o["q_draft"], ws)
 
-    def barrier():
-        if dist is not None:
-            dist.barrier()
+    barrier = shard.barrier
 
-    for c in range(args.warmup):
-        step(c)
-    st = sd.sync_status(ws)
-    if st != sd.SPEC_OK:
-        raise RuntimeError(f"device status {sd.status_string(st)}")
-    taus = []
-    barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
+        for c in range(args.warmup):
+            step(c)
+        st = sd.sync_status(ws)
+        if st != sd.SPEC_OK:
+            raise RuntimeError(f"device status {sd.status_string(st)}")
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        clk.mark_start()
         e0.record(stream)
         for c in range(args.steps):
             step(args.warmup + c)
         e1.record(stream)
         torch.cuda.synchronize()
-    barrier()
+        clk.mark_end()
+        barrier()
     ms = e0.elapsed_time(e1)
     launches = args.steps  # one fused kernel per cycle
     st = sd.sync_status(ws)
     if st != sd.SPEC_OK:
         raise RuntimeError(f"device status {sd.status_string(st)}")
     tau = o["tau"].cpu().numpy()
-    ms_t = torch.tensor([ms], device=dev)
-    if dist is not None:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = shard.max_over_ranks(ms)
     per_step_ms = ms_max / args.steps
-    positions = w.B * w.K * world * args.steps
+    positions = shard.sum_over_ranks(p.B * w.K * args.steps)
     value = positions / (ms_max / 1e3)
 
     # end to end through the C-ABI with host buffers: pinned H2D of the step's
@@ -281,10 +289,8 @@ def run_ours(args, rank, world, local_rank):
         e2e_step(10_000 + c)
     f1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([f0.elapsed_time(f1)], device=dev)
-    if dist is not None:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_value = w.B * w.K * world * e2e_steps / (float(e2e_ms.item()) / 1e3)
+    e2e_ms = shard.max_over_ranks(f0.elapsed_time(f1))
+    e2e_value = shard.sum_over_ranks(p.B * w.K * e2e_steps) / (e2e_ms / 1e3)
     h2d = hbase.numel() * hbase.element_size() + htarget.numel() * htarget.element_size() + \
         hlast.numel() * hlast.element_size()
     d2h = hout.numel() * hout.element_size() + htau.numel() * htau.element_size()
@@ -306,6 +312,7 @@ def run_ours(args, rank, world, local_rank):
                        "l2": "logit inputs 546 MB > L2; W L2-resident by design",
                        "mean_tau": float(tau.mean())},
             "gpu_launches": launches * world,
+            "rows_per_rank": p.B,
             "hbm_gbs_full_stream": achieved,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": recorded_traffic(h),
@@ -318,9 +325,10 @@ def run_ours(args, rank, world, local_rank):
                     "d2h_bytes_per_step": d2h},
         }
         if world == 1:
-            line["cpu_baseline"] = cpu_baseline(w, d)
+            line["cpu_baseline"] = None if args.no_cpu_baseline else cpu_baseline(w, d)
         print(json.dumps(line), flush=True)
-    if dist is not None:
+    if multi:
+        import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
 
@@ -328,8 +336,10 @@ def run_ours(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the timed oracle sample (profiling runs)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     args = ap.parse_args()
     if args.warmup < 3:

@@ -77,18 +77,22 @@ bool make_tmap_W(CUtensorMap* m, const void* W, int r, int V) {
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_tmap_base(CUtensorMap* m, const void* base, int dtype, int B, int K, int V, int N) {
+// Base logits [B, K, V] as a 3-D map.  Tensor-core path: boxes of 64 tokens x
+// 1 step x N rows with the 128-byte swizzle, the operand layout the bias MMA
+// adds them with; otherwise 128 tokens x 1 x N rows, unswizzled.
+bool make_tmap_base(CUtensorMap* m, const void* base, int dtype, int B, int K, int V, int N,
+                    bool tc) {
   EncodeTiledFn f = encode_fn();
   if (!f) return false;
   const size_t es = dtype == SPEC_BF16 ? 2 : 4;
   const cuuint64_t dims[3] = {(cuuint64_t)V, (cuuint64_t)K, (cuuint64_t)B};
   const cuuint64_t strides[2] = {(cuuint64_t)V * es, (cuuint64_t)K * V * es};
-  const cuuint32_t box[3] = {128, 1, (cuuint32_t)N};
+  const cuuint32_t box[3] = {tc ? 64u : 128u, 1, (cuuint32_t)N};
   const cuuint32_t estr[3] = {1, 1, 1};
   return f(m, dtype == SPEC_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
            3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-           CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+           tc ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // ---- debug kernels: Philox stream and the CUDA library's own Philox4_32_10 ----
@@ -236,7 +240,7 @@ static spec_status run_cycle(const spec_params* p, int mode, const void* base, c
   CUtensorMap tmW, tmBase;
   memset(&tmW, 0, sizeof(tmW));
   if (g.tc && !make_tmap_W(&tmW, W, p->r, p->V)) return SPEC_ERR_CUDA;
-  if (!make_tmap_base(&tmBase, base, p->dtype, p->B, p->K, p->V, g.N)) return SPEC_ERR_CUDA;
+  if (!make_tmap_base(&tmBase, base, p->dtype, p->B, p->K, p->V, g.N, g.tc)) return SPEC_ERR_CUDA;
   CycleLaunch L;
   L.base = base;
   L.target = target;

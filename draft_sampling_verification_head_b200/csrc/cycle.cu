@@ -348,7 +348,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
   uint8_t* sU = sW + (TC ? (size_t)kNS * kWStage : 0);              // TC: nkb x N x 128 B
   float* sUf = reinterpret_cast<float*>(sU);                        // FMA: N x r floats
   const size_t u_bytes = TC ? (size_t)nkb * N * 128 : (size_t)N * a.r * 4;
-  T* sBase = reinterpret_cast<T*>(sU + ((u_bytes + 1023) & ~size_t(1023)));  // kNBS x N x 128
+  // TC: N x N identity (B operand, K-major, 128-byte swizzle) that makes the
+  // MMA add each base tile to the bias
+  uint8_t* sI = sU + ((u_bytes + 1023) & ~size_t(1023));
+  T* sBase = reinterpret_cast<T*>(sI + (TC ? (size_t)N * 128 : 0));  // kNBS x N x 128 tokens
   const size_t base_bytes = (size_t)kNBS * N * kCH * sizeof(T);
   float2* sBucket = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(sBase) + base_bytes);
   float* zbuf = reinterpret_cast<float*>(sBucket);  // owner staging, after the bucket walk
@@ -381,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
     }
     for (int i = 0; i < kNBS; ++i) {
       mbar_init(&ctl->bfull[i], 1);
-      mbar_init(&ctl->bempty[i], kComputeThreads / 32);
+      mbar_init(&ctl->bempty[i], TC ? 1 : kComputeThreads / 32);  // TC: freed by the MMA
     }
     for (int i = 0; i < kMaxNC; ++i) mbar_init(&ctl->dfull[i], 1);
     mbar_init(&ctl->bready, 1);
@@ -393,6 +396,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
   if (warp == 0) {
     tmem_alloc(&ctl->tmem_slot, ncols);
     tmem_relinquish();
+  }
+  if (TC) {  // identity I[n][k] = (n == k), k < 64, rows of 128 bytes, 16-byte chunks swizzled
+    for (int idx = tid; idx < N * 64; idx += kThreads) {
+      const int n = idx >> 6, kk = idx & 63;
+      reinterpret_cast<__nv_bfloat16*>(sI + n * 128 + (((kk >> 3) ^ (n & 7)) << 4))[kk & 7] =
+          __float2bfloat16(n == kk ? 1.f : 0.f);
+    }
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -455,8 +466,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               break;
             }
             mbar_arrive_expect_tx(&ctl->bfull[slot], (uint32_t)(N * kCH * sizeof(T)));
-            tma_load_3d(sBase + (size_t)slot * N * kCH, &a.tmBase, &ctl->bfull[slot],
-                        (chunk0 + cl) * kCH, s, g * N, polB);
+            if (TC) {  // [N][64] per half: tokens 0..63, then 64..127
+              tma_load_3d(sBase + (size_t)slot * N * kCH, &a.tmBase, &ctl->bfull[slot],
+                          (chunk0 + cl) * kCH, s, g * N, polB);
+              tma_load_3d(sBase + (size_t)slot * N * kCH + N * 64, &a.tmBase, &ctl->bfull[slot],
+                          (chunk0 + cl) * kCH + 64, s, g * N, polB);
+            } else {
+              tma_load_3d(sBase + (size_t)slot * N * kCH, &a.tmBase, &ctl->bfull[slot],
+                          (chunk0 + cl) * kCH, s, g * N, polB);
+            }
             ++Lb;
           }
         }
@@ -471,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
   else if (warp == kMmaWarp) {
     if (TC && lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, N, /*a_mn_major=*/true, /*b_mn_major=*/false);
-      uint32_t Lw = 0, step_ctr = 0;
+      uint32_t Lw = 0, Lb = 0, step_ctr = 0;
       bool ok = true;
       for (int g = 0; g < a.ngroups && ok; ++g) {
         for (int s = 0; s < nsteps && ok; ++s, ++step_ctr) {
@@ -509,7 +527,30 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               umma_commit(&ctl->wempty[slot]);
               ++Lw;
             }
+            // z = bias + base: D += base^T (M = tokens, K = batch rows, MN-major)
+            // x I (K-major), exact in fp32 since every product is base x 1 or x 0
+            if (ok && s < K) {
+              const uint32_t bslot = Lb % kNBS;
+              if (!mbar_wait_bounded(&ctl->bfull[bslot], (Lb / kNBS) & 1, a.spin, &hdr->abort)) {
+                record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_BASE, cta, s);
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t a_base = smem_u32(sBase + (size_t)bslot * N * kCH);
+              const uint32_t b_base = smem_u32(sI);
+#pragma unroll
+              for (int kk = 0; kk < N / 16; ++kk) {
+                const uint64_t ad = smem_desc_sw128(a_base + kk * 2048, N * 128, 1024);
+                const uint64_t bd = smem_desc_sw128(b_base + kk * 32, 16, 1024);
+                umma_bf16(dcol, ad, bd, idesc, 1u);
+              }
+              umma_commit(&ctl->bempty[bslot]);
+              ++Lb;
+            }
             if (ok) umma_commit(&ctl->dfull[cl]);
+            if (a.trace && cta == 0 && g == 0 && cl < 8)
+              a.trace[(size_t)min(s, K) * kTracePhases + 24 + cl] = globaltimer_ns();
           }
           if (a.trace && cta == 0 && g == 0) a.trace[(size_t)min(s, K) * kTracePhases + 10] = globaltimer_ns();
         }
@@ -1028,7 +1069,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
         bool fast = !a.greedy && i > 0;
         for (int attempt = 0; attempt < 2; ++attempt) {
           // ---------------- epilogue: z = base + bias, bucket statistics
-          uint64_t t_wait = 0;
+          uint64_t t_wait = 0, t_base = 0, t_st = 0;
           float rmax[NCOL];
 #pragma unroll
           for (int j = 0; j < NCOL; ++j) rmax[j] = -INFINITY;
@@ -1040,18 +1081,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             const uint32_t tcol = taddr + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(cl * N + n0);
             if (attempt == 0) {
               const uint64_t t_w0 = trace ? globaltimer_ns() : 0;
-              bias_tile(cl, d);
+              bias_tile(cl, d);  // TC: already z = bias + base, added by the MMA
               if (trace) t_wait += globaltimer_ns() - t_w0;
-              const uint32_t bslot = Lb % kNBS;
-              if (!mbar_wait_bounded(&ctl->bfull[bslot], (Lb / kNBS) & 1, a.spin, &hdr->abort))
-                soft_fail(SPEC_ERR_TIMEOUT, SITE_MBAR_BASE, cta, i);
-              const T* bt = sBase + (size_t)bslot * N * kCH;
+              if (!TC) {
+                const uint32_t bslot = Lb % kNBS;
+                const uint64_t t_b0 = trace ? globaltimer_ns() : 0;
+                if (!mbar_wait_bounded(&ctl->bfull[bslot], (Lb / kNBS) & 1, a.spin, &hdr->abort))
+                  soft_fail(SPEC_ERR_TIMEOUT, SITE_MBAR_BASE, cta, i);
+                if (trace) t_base += globaltimer_ns() - t_b0;
+                const T* bt = sBase + (size_t)bslot * N * kCH;
 #pragma unroll
-              for (int j = 0; j < NCOL; ++j)
-                d[j] = valid ? d[j] + to_f<T>(bt[(n0 + j) * kCH + vl]) : -INFINITY;
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&ctl->bempty[bslot]);
-              ++Lb;
+                for (int j = 0; j < NCOL; ++j) d[j] += to_f<T>(bt[(n0 + j) * kCH + vl]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->bempty[bslot]);
+                ++Lb;
+              }
+#pragma unroll
+              for (int j = 0; j < NCOL; ++j) d[j] = valid ? d[j] : -INFINITY;
               if (a.biased_out && valid) {
 #pragma unroll
                 for (int j = 0; j < NCOL; ++j) {
@@ -1060,9 +1106,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
                 }
               }
               // z replaces the bias in tensor memory: owner scans (and a redo) read it
-              if (!a.greedy) tmem_st_cols<NCOL>(tcol, d);
+              const uint64_t t_s0 = trace ? globaltimer_ns() : 0;
+              if (!TC && !a.greedy) tmem_st_cols<NCOL>(tcol, d);  // TC: z is in tensor memory
+              if (trace) t_st += globaltimer_ns() - t_s0;
             } else {
               tmem_ld_cols<NCOL>(tcol, d);  // z of this step, kept in tensor memory
+#pragma unroll
+              for (int j = 0; j < NCOL; ++j) d[j] = valid ? d[j] : -INFINITY;
             }
             float2* bk = sBucket + ((size_t)cl * 4 + q4) * N;
             constexpr int REP = 32 / NCOL;
@@ -1088,6 +1138,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               bfly_ms<NCOL>(d, s, k, lane);
               if ((lane & (REP - 1)) == 0) bk[n0 + lane / REP] = make_float2(d[0], s[0]);
             }
+            if (trace && g == 0 && cl < 8 && attempt == 0)
+              trace[(size_t)i * kTracePhases + 16 + cl] = globaltimer_ns();
           }
           if (fast) {  // true max of z per row over this warp's tokens
             bfly_max1<NCOL>(rmax, lane);
@@ -1097,7 +1149,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           named_sync();
           tc_fence_after();
           mark(g, i, 2);
-          if (trace && g == 0) trace[(size_t)i * kTracePhases + 11] = t_wait;
+          if (trace && g == 0) {
+            trace[(size_t)i * kTracePhases + 11] = t_wait;
+            trace[(size_t)i * kTracePhases + 13] = t_base;
+            trace[(size_t)i * kTracePhases + 14] = t_st;
+          }
           // ---------------- CTA partial per batch row (TPB threads per row)
           {
             const int n = grp_n;
@@ -1506,6 +1562,7 @@ size_t smem_bytes(int r, int nc) {
   if (TC) s += (size_t)kNS * kWStage;
   const size_t u = TC ? (size_t)nkb * N * 128 : (size_t)N * r * 4;
   s += (u + 1023) & ~size_t(1023);
+  if (TC) s += (size_t)N * 128;  // identity operand
   s += (size_t)kNBS * N * kCH * sizeof(T);
   s += bucket_region_bytes(nc, N);
   s += sizeof(Ctl<N>);

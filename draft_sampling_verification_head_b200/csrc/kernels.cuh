@@ -55,7 +55,7 @@ struct CycleGeom {
 bool cycle_geometry(int B, int K, int V, int r, int dtype, uint32_t flags, int num_sms,
                     CycleGeom* g, const char** why);
 size_t cycle_ws_bytes(int K, const CycleGeom& g);
-constexpr int kTracePhases = 16;  // timeline slots per step
+constexpr int kTracePhases = 32;  // timeline slots per step
 size_t cycle_trace_bytes(int K);
 
 struct CycleLaunch {
@@ -82,7 +82,8 @@ cudaError_t launch_cycle(const CycleLaunch& L, const CycleGeom& g, WsHeader* hdr
 
 // ---- Tensor maps --------------------------------------------------------------
 bool make_tmap_W(CUtensorMap* m, const void* W, int r, int V);
-bool make_tmap_base(CUtensorMap* m, const void* base, int dtype, int B, int K, int V, int N);
+bool make_tmap_base(CUtensorMap* m, const void* base, int dtype, int B, int K, int V, int N,
+                    bool tc);
 
 // ---- Debug ------------------------------------------------------------------------
 cudaError_t launch_debug_philox(const uint32_t* ctr, const uint32_t* key, uint32_t* out, int n,

@@ -80,11 +80,12 @@ typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 #define SPEC_FLAG_FMA_BIAS 1u  /* compute the Markov bias with fp32 FMAs instead of tensor cores */
 #define SPEC_FLAG_TRACE 2u     /* spec_cycle / spec_markov_bias_sample: record a device timeline.
                                   CTA 0 writes %globaltimer (ns) into the workspace at byte offset
-                                  256 as uint64 [K+2][16]: row i < K = draft step i (slots: 0 start,
+                                  256 as uint64 [K+2][32]: row i < K = draft step i (slots: 0 start,
                                   1 rows gathered, 2 epilogue done, 3 partials published, 4 target
                                   rows streamed, 5 barrier passed, 6 partials combined, 7 owner
-                                  draws done, 8 tokens known), row K = final step, row K+1 =
-                                  prologue.  Only the first batch group is recorded. */
+                                  draws done, 8 tokens known; 9..31 finer diagnostics: tensor-core
+                                  issue, wait totals, per-chunk times), row K = final step, row
+                                  K+1 = prologue.  Only the first batch group is recorded. */
 
 typedef struct {
   int32_t B;             /* batch rows, >= 1 */

@@ -213,6 +213,16 @@ SPEC_DEV void tma_load_2d(void* dst, const CUtensorMap* m, uint64_t* bar, int32_
       "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
+// Untiled bulk copy global -> this CTA's shared memory, completion counted in
+// bytes on the mbarrier.  Both addresses 16-byte aligned, bytes a multiple of 16.
+SPEC_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                        uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
 SPEC_DEV void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int32_t x, int32_t y,
                           int32_t z, uint64_t policy) {
   asm volatile(

@@ -86,7 +86,8 @@ struct Args {
 template <int N>
 struct Ctl {
   uint64_t wfull[kNS], wempty[kNS], bfull[kNBS], bempty[kNBS], dfull[kMaxNC];
-  uint64_t bready, tfree, mmadone;
+  uint64_t ffull[kNBS], fempty[kNBS];  // final step: gathered stop-row tiles in the base ring
+  uint64_t bready, tfree, mmadone, rows_known;
   uint32_t tmem_slot;
   int32_t abort_local;
   int32_t n_owned;
@@ -101,6 +102,7 @@ struct Ctl {
   float zM[N], zS[N];   // draft stats of the stop row
   float Mt[N], St[N];   // target stats of row i during a step
   float fMt[N], fSt[N]; // target stats of the final row (stop row or row K)
+  float rfSt[N], rzS[N]; // 1 / fSt and 1 / zS for the final step
   float ref[N];         // per-row reference of the fast path (previous step's max)
   float cmax[4][N];     // true max per row and tensor-memory quadrant
   int32_t redo;
@@ -386,7 +388,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
       mbar_init(&ctl->bfull[i], 1);
       mbar_init(&ctl->bempty[i], TC ? 1 : kComputeThreads / 32);  // TC: freed by the MMA
     }
+    for (int i = 0; i < kNBS; ++i) {
+      mbar_init(&ctl->ffull[i], 1);
+      mbar_init(&ctl->fempty[i], kComputeThreads / 32);
+    }
     for (int i = 0; i < kMaxNC; ++i) mbar_init(&ctl->dfull[i], 1);
+    mbar_init(&ctl->rows_known, 1);
     mbar_init(&ctl->bready, 1);
     mbar_init(&ctl->tfree, 1);
     mbar_init(&ctl->mmadone, 1);
@@ -449,38 +456,84 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
         mbar_drain(&ctl->wfull[L % kNS], (L / kNS) & 1);
     }
   } else if (warp == kBaseWarp) {
-    if (lane == 0) {
-      const uint64_t polB = policy_evict_first();
-      tma_prefetch_desc(&a.tmBase);
-      uint32_t Lb = 0;
-      bool ok = true;
-      for (int g = 0; g < a.ngroups && ok; ++g) {
-        for (int s = 0; s < K && ok; ++s) {
-          for (int cl = 0; cl < ncc; ++cl) {
-            const uint32_t slot = Lb % kNBS;
-            if (Lb >= kNBS &&
-                !mbar_wait_bounded(&ctl->bempty[slot], ((Lb / kNBS) - 1) & 1, a.spin,
-                                   &hdr->abort)) {
-              record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_BASE, cta, s);
-              ok = false;
-              break;
-            }
+    // Draft steps: one base tile [N rows x 128 tokens] per chunk and step, by
+    // lane 0 through the tensor map.  Final step (stochastic cycle): for each
+    // chunk a target tile and a base tile of the rows' stop rows (row K for a
+    // row that accepted every draft), gathered row by row with bulk copies by
+    // all 32 lanes once the stop rows are known.
+    const uint64_t polB = policy_evict_first();
+    if (lane == 0) tma_prefetch_desc(&a.tmBase);
+    uint32_t Lb = 0, Lf = 0;
+    int ok = 1;
+    auto wait0 = [&](uint64_t* bar, uint32_t parity, int where) {  // lane 0 waits, all learn
+      int r = 1;
+      if (lane == 0 && !mbar_wait_bounded(bar, parity, a.spin, &hdr->abort)) {
+        record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_BASE, cta, where);
+        r = 0;
+      }
+      return __shfl_sync(FULL, r, 0);
+    };
+    for (int g = 0; g < a.ngroups && ok; ++g) {
+      // slots last held final-step tiles of the previous group: wait until read
+      for (uint32_t L = (Lf > kNBS ? Lf - kNBS : 0); L < Lf && ok; ++L)
+        ok = wait0(&ctl->fempty[L % kNBS], (L / kNBS) & 1, 2000 + g);
+      for (int s = 0; s < K && ok; ++s) {
+        for (int cl = 0; cl < ncc && ok; ++cl) {
+          const uint32_t slot = Lb % kNBS;
+          if (Lb >= kNBS) ok = wait0(&ctl->bempty[slot], ((Lb / kNBS) - 1) & 1, s);
+          if (!ok) break;
+          if (lane == 0) {
             mbar_arrive_expect_tx(&ctl->bfull[slot], (uint32_t)(N * kCH * sizeof(T)));
             if (TC) {  // [N][64] per half: tokens 0..63, then 64..127
               tma_load_3d(sBase + (size_t)slot * N * kCH, &a.tmBase, &ctl->bfull[slot],
                           (chunk0 + cl) * kCH, s, g * N, polB);
-              tma_load_3d(sBase + (size_t)slot * N * kCH + N * 64, &a.tmBase, &ctl->bfull[slot],
-                          (chunk0 + cl) * kCH + 64, s, g * N, polB);
+              tma_load_3d(sBase + (size_t)slot * N * kCH + N * 64, &a.tmBase,
+                          &ctl->bfull[slot], (chunk0 + cl) * kCH + 64, s, g * N, polB);
             } else {
               tma_load_3d(sBase + (size_t)slot * N * kCH, &a.tmBase, &ctl->bfull[slot],
                           (chunk0 + cl) * kCH, s, g * N, polB);
             }
-            ++Lb;
           }
+          ++Lb;
         }
       }
+      if (!has_final || !ok) continue;
+      // every draft tile read, stop rows of this group known
+      for (uint32_t L = (Lb > kNBS ? Lb - kNBS : 0); L < Lb && ok; ++L)
+        ok = wait0(&ctl->bempty[L % kNBS], (L / kNBS) & 1, 1000 + g);
+      if (ok) ok = wait0(&ctl->rows_known, (uint32_t)g & 1, 3000 + g);
+      const int nb_g = min(N, a.B - g * N);
+      for (int cl = 0; cl < ncc && ok; ++cl) {
+        const int v0 = (chunk0 + cl) * kCH;
+        const uint32_t bytes = (uint32_t)(min(kCH, V - v0) * sizeof(T));
+        for (int t = 0; t < 2 && ok; ++t) {  // t = 0: target rows, t = 1: base rows
+          const uint32_t slot = Lf % kNBS;
+          if (Lf >= kNBS) ok = wait0(&ctl->fempty[slot], ((Lf / kNBS) - 1) & 1, 4000 + cl);
+          if (!ok) break;
+          int rows = 0;
+          for (int n = 0; n < nb_g; ++n) rows += (t == 0 || !ctl->alive[n]) ? 1 : 0;
+          if (lane == 0) mbar_arrive_expect_tx(&ctl->ffull[slot], (uint32_t)rows * bytes);
+          __syncwarp();
+          T* dst = sBase + (size_t)slot * N * kCH;
+          for (int n = lane; n < nb_g; n += 32) {
+            const bool alive = ctl->alive[n] != 0;
+            if (t == 1 && alive) continue;
+            const int row = alive ? K : ctl->stoprow[n];
+            const int64_t b = (int64_t)g * N + n;
+            const T* src = t == 0 ? target + (b * (K + 1) + row) * V + v0
+                                  : base + (b * K + row) * V + v0;
+            bulk_load(dst + (size_t)n * kCH, src, bytes, &ctl->ffull[slot], polB);
+          }
+          ++Lf;
+        }
+      }
+    }
+    // nothing in flight at exit: the latest copy into every slot has landed
+    if (lane == 0) {
       for (uint32_t L = (Lb > kNBS ? Lb - kNBS : 0); L < Lb; ++L)
         mbar_drain(&ctl->bfull[L % kNBS], (L / kNBS) & 1);
+      for (uint32_t L = (Lf > kNBS ? Lf - kNBS : 0); L < Lf; ++L)
+        mbar_drain(&ctl->ffull[L % kNBS], (L / kNBS) & 1);
     }
   }
   // =========================================================================
@@ -565,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
   else {
     const int q4 = warp & 3;         // tensor-memory lane quadrant
     const int n0 = (warp >> 2) * NCOL;  // first column (batch row) of this warp
-    uint32_t step_ctr = 0, Lb = 0;
+    uint32_t step_ctr = 0, Lb = 0, Lf = 0;
     uint32_t nbar = 0, tok_expected = 0, rec_expected = 0;
     // Failures are folded into the CTA-wide flag ctl->abort_local; it is only
     // read right after a named barrier, so every compute thread takes the same
@@ -1353,6 +1406,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
         }
       }  // draft steps
       if (failed) break;
+      // alive / stoprow are final: the producer may gather the stop rows
+      if (has_final && tid == 0) mbar_arrive(&ctl->rows_known);
 
       if (a.mode == MODE_CYCLE) {
         // row-K target partials (written after the last barrier) become visible
@@ -1391,6 +1446,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               if (p < 0 || p >= V) p = 0;
             }
             ctl->prev[n] = p;
+            if (n < nb_g) {
+              ctl->rfSt[n] = 1.f / ctl->fSt[n];
+              ctl->rzS[n] = ctl->alive[n] ? 0.f : 1.f / ctl->zS[n];
+            }
           }
           named_sync();
           gather_u(nb_g);
@@ -1400,15 +1459,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             bias_tile(cl, d);
             const int v = (chunk0 + cl) * kCH + q4 * 32 + lane;
             const bool valid = v < V;
+            // gathered stop-row tiles (entries past the copied rows / tokens are
+            // stale and only read under the guards below)
             float tv[NCOL], bvv[NCOL];
+            {
+              const uint32_t ts = Lf % kNBS, bs = (Lf + 1) % kNBS;
+              if (!mbar_wait_bounded(&ctl->ffull[ts], (Lf / kNBS) & 1, a.spin, &hdr->abort) ||
+                  !mbar_wait_bounded(&ctl->ffull[bs], ((Lf + 1) / kNBS) & 1, a.spin, &hdr->abort))
+                soft_fail(SPEC_ERR_TIMEOUT, SITE_MBAR_BASE, cta, 5000 + cl);
+              const T* tt = sBase + (size_t)ts * N * kCH;
+              const T* bt = sBase + (size_t)bs * N * kCH;
+              const int vl = q4 * 32 + lane;
 #pragma unroll
-            for (int j = 0; j < NCOL; ++j) {  // loads from clamped valid addresses
-              const int n = min(n0 + j, nb_g - 1);
-              const int b = g * N + n;
-              const int row = ctl->alive[n] ? K : ctl->stoprow[n];
-              const int vv = valid ? v : V - 1;
-              tv[j] = ld_elem(target, ((int64_t)b * (K + 1) + row) * V + vv);
-              bvv[j] = ld_elem(base, ((int64_t)b * K + min(row, K - 1)) * V + vv);
+              for (int j = 0; j < NCOL; ++j) {
+                tv[j] = to_f<T>(tt[(n0 + j) * kCH + vl]);
+                bvv[j] = to_f<T>(bt[(n0 + j) * kCH + vl]);
+              }
+              __syncwarp();
+              if (lane == 0) {
+                mbar_arrive(&ctl->fempty[ts]);
+                mbar_arrive(&ctl->fempty[bs]);
+              }
+              Lf += 2;
             }
             // residual mass r (into tv) and target mass p (into bvv), in place
 #pragma unroll
@@ -1416,10 +1488,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               const int n = n0 + j;
               float r = 0.f, p = 0.f;
               if (valid && n < nb_g) {
-                p = exp2f((tv[j] - ctl->fMt[n]) * k) / ctl->fSt[n];
+                p = exp2f((tv[j] - ctl->fMt[n]) * k) * ctl->rfSt[n];
                 r = p;
                 if (!ctl->alive[n])
-                  r = fmaxf(p - exp2f((d[j] + bvv[j] - ctl->zM[n]) * k) / ctl->zS[n], 0.f);
+                  r = fmaxf(p - exp2f((d[j] + bvv[j] - ctl->zM[n]) * k) * ctl->rzS[n], 0.f);
               }
               tv[j] = r;
               bvv[j] = p;
@@ -1499,10 +1571,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               const int v = v0 + lane;
               float w = 0.f;
               if (v < V) {
-                const float p = exp2f((tvv[j] - ctl->fMt[n]) * k) / ctl->fSt[n];
+                const float p = exp2f((tvv[j] - ctl->fMt[n]) * k) * ctl->rfSt[n];
                 w = p;
                 if (!bonus && !use_p)
-                  w = fmaxf(p - exp2f((dv[j] + bvv[j] - ctl->zM[n]) * k) / ctl->zS[n], 0.f);
+                  w = fmaxf(p - exp2f((dv[j] + bvv[j] - ctl->zM[n]) * k) * ctl->rzS[n], 0.f);
               }
               const int wl = bucket_scan(w, ctl->obtarget[oo[j]]);
               if (lane == 0) a.out[(int64_t)b * (K + 1) + row] = v0 + wl;

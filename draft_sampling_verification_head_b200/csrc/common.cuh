@@ -352,6 +352,16 @@ SPEC_DEV float warp_max(float v) {
   return v;
 }
 
+// 2^x by the hardware approximation (PTX ex2.approx.ftz.f32, a few ulp of
+// relative error); results below 2^-126 flush to zero.  Every exponential of the
+// fused cycle goes through this one function, so a quantity computed in two
+// places (a bucket total and the scan inside the bucket) agrees bit for bit.
+SPEC_DEV float fexp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Softmax statistics are kept as (m, s): m = max of the raw logits x,
 // s = sum exp2((x - m) * k) with k = log2(e) / T.  Differences x - m are taken
 // before scaling so that the dominant terms carry no rounding from the scale.
@@ -361,7 +371,7 @@ SPEC_DEV void ms_combine(float& m, float& s, float m2, float s2, float k) {
   const bool first = m >= m2;
   const float mb = first ? m : m2, ml = first ? m2 : m;
   const float sb = first ? s : s2, sl = first ? s2 : s;
-  const float e = (ml == -INFINITY) ? 0.f : exp2f((ml - mb) * k);
+  const float e = (ml == -INFINITY) ? 0.f : fexp2((ml - mb) * k);
   m = mb;
   s = fmaf(sl, e, sb);
 }

@@ -50,6 +50,7 @@ constexpr int kMmaWarp = 9;
 constexpr int kBaseWarp = 10;
 constexpr int kNS = 6;              // W ring stages
 constexpr int kNBS = 4;             // base tile ring stages
+constexpr int kIL = 1;              // chunks whose MMA chains are interleaved
 constexpr int kMaxNC = 32;
 constexpr int kWStage = kCH * 64 * 2;  // 16 KB: 128 tokens x 64 rank, bf16
 constexpr int kMaxG = 160;          // CTAs a launch may use (>= SM count); partial-row stride
@@ -103,6 +104,7 @@ struct Ctl {
   float Mt[N], St[N];   // target stats of row i during a step
   float fMt[N], fSt[N]; // target stats of the final row (stop row or row K)
   float rfSt[N], rzS[N]; // 1 / fSt and 1 / zS for the final step
+  float uacc[N];        // accept-test uniform of the current step
   float ref[N];         // per-row reference of the fast path (previous step's max)
   float cmax[4][N];     // true max per row and tensor-memory quadrant
   int32_t redo;
@@ -138,6 +140,15 @@ SPEC_DEV Rec load_rec(const Rec* src) {
   d4[1] = __ldcg(s4 + 1);
   d4[2] = __ldcg(s4 + 2);
   return r;
+}
+
+// Shared region of the MMA's U operand (tensor cores: bf16 rows in k-blocks;
+// otherwise fp32 rows), reused for the owners' staged logits.
+template <typename T, bool TC, int N>
+__host__ __device__ inline size_t u_region_bytes(int r) {
+  const size_t u = TC ? (size_t)(r / 64) * N * 128 : (size_t)N * r * 4;
+  const size_t st = (size_t)2 * N * 32 * sizeof(T);
+  return u > st ? u : st;
 }
 
 // Shared region for per-bucket statistics, reused to stage owned rows' values.
@@ -349,7 +360,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
   uint8_t* sW = smem;                                               // TC: kNS x 16 KB
   uint8_t* sU = sW + (TC ? (size_t)kNS * kWStage : 0);              // TC: nkb x N x 128 B
   float* sUf = reinterpret_cast<float*>(sU);                        // FMA: N x r floats
-  const size_t u_bytes = TC ? (size_t)nkb * N * 128 : (size_t)N * a.r * 4;
+  const size_t u_bytes = u_region_bytes<T, TC, N>(a.r);
+  // Owner staging of the chosen buckets' logits: overlays the U operand,
+  // which nothing reads between a step's last MMA and the next gather.
+  T* tbuf = reinterpret_cast<T*>(sU);
+  T* bbuf = tbuf + N * 32;
   // TC: N x N identity (B operand, K-major, 128-byte swizzle) that makes the
   // MMA add each base tile to the bias
   uint8_t* sI = sU + ((u_bytes + 1023) & ~size_t(1023));
@@ -430,23 +445,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
       bool ok = true;
       for (int g = 0; g < a.ngroups && ok; ++g) {
         for (int s = 0; s < nsteps && ok; ++s) {
-          for (int cl = 0; cl < ncc && ok; ++cl) {
-            const int v0 = (chunk0 + cl) * kCH;
-            for (int kb = 0; kb < nkb; ++kb) {
-              const uint32_t slot = Lw % kNS;
-              if (Lw >= kNS &&
-                  !mbar_wait_bounded(&ctl->wempty[slot], ((Lw / kNS) - 1) & 1, a.spin,
-                                     &hdr->abort)) {
-                record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_FULL, cta, 100 + s);
-                ok = false;
-                break;
+          // stages in the MMA's order: k-block by k-block over kIL chunks at a time
+          for (int c0 = 0; c0 < ncc && ok; c0 += kIL) {
+            const int nil = min(kIL, ncc - c0);
+            for (int kb = 0; kb < nkb && ok; ++kb) {
+              for (int c = 0; c < nil; ++c) {
+                const int v0 = (chunk0 + c0 + c) * kCH;
+                const uint32_t slot = Lw % kNS;
+                if (Lw >= kNS &&
+                    !mbar_wait_bounded(&ctl->wempty[slot], ((Lw / kNS) - 1) & 1, a.spin,
+                                       &hdr->abort)) {
+                  record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_FULL, cta, 100 + s);
+                  ok = false;
+                  break;
+                }
+                mbar_arrive_expect_tx(&ctl->wfull[slot], kWStage);
+                tma_load_2d(sW + (size_t)slot * kWStage, &a.tmW, &ctl->wfull[slot], v0, kb * 64,
+                            polW);
+                tma_load_2d(sW + (size_t)slot * kWStage + kWStage / 2, &a.tmW,
+                            &ctl->wfull[slot], v0 + 64, kb * 64, polW);
+                ++Lw;
               }
-              mbar_arrive_expect_tx(&ctl->wfull[slot], kWStage);
-              tma_load_2d(sW + (size_t)slot * kWStage, &a.tmW, &ctl->wfull[slot], v0, kb * 64,
-                          polW);
-              tma_load_2d(sW + (size_t)slot * kWStage + kWStage / 2, &a.tmW, &ctl->wfull[slot],
-                          v0 + 64, kb * 64, polW);
-              ++Lw;
             }
           }
         }
@@ -559,51 +578,74 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           }
           tc_fence_after();
           if (a.trace && cta == 0 && g == 0) a.trace[(size_t)min(s, K) * kTracePhases + 9] = globaltimer_ns();
-          for (int cl = 0; cl < ncc && ok; ++cl) {
-            const uint32_t dcol = taddr + (uint32_t)(cl * N);
-            for (int kb = 0; kb < nkb; ++kb) {
-              const uint32_t slot = Lw % kNS;
-              if (!mbar_wait_bounded(&ctl->wfull[slot], (Lw / kNS) & 1, a.spin, &hdr->abort)) {
-                record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_FULL, cta, s);
-                ok = false;
-                break;
+          // kIL chunks at a time, their MMAs alternating: each chunk's K-steps
+          // accumulate into its own columns, so the chains overlap in the pipe
+          for (int c0 = 0; c0 < ncc && ok; c0 += kIL) {
+            const int nil = min(kIL, ncc - c0);
+            for (int kb = 0; kb < nkb && ok; ++kb) {
+              uint32_t a_base[kIL];
+              for (int c = 0; c < nil; ++c) {
+                const uint32_t slot = (Lw + c) % kNS;
+                if (!mbar_wait_bounded(&ctl->wfull[slot], ((Lw + c) / kNS) & 1, a.spin,
+                                       &hdr->abort)) {
+                  record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_FULL, cta, s);
+                  ok = false;
+                  break;
+                }
+                a_base[c] = smem_u32(sW + (size_t)slot * kWStage);
               }
+              if (!ok) break;
               tc_fence_after();
-              const uint32_t a_base = smem_u32(sW + (size_t)slot * kWStage);
               const uint32_t b_base = smem_u32(sU + (size_t)kb * N * 128);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t ad = smem_desc_sw128(a_base + kk * 2048, 8192, 1024);
                 const uint64_t bd = smem_desc_sw128(b_base + kk * 32, 16, 1024);
-                umma_bf16(dcol, ad, bd, idesc, (kb | kk) != 0);
+#pragma unroll
+                for (int c = 0; c < kIL; ++c) {
+                  if (c >= nil) break;
+                  const uint64_t ad = smem_desc_sw128(a_base[c] + kk * 2048, 8192, 1024);
+                  umma_bf16(taddr + (uint32_t)((c0 + c) * N), ad, bd, idesc, (kb | kk) != 0);
+                }
               }
-              umma_commit(&ctl->wempty[slot]);
-              ++Lw;
+              for (int c = 0; c < nil; ++c) umma_commit(&ctl->wempty[(Lw + c) % kNS]);
+              Lw += nil;
             }
             // z = bias + base: D += base^T (M = tokens, K = batch rows, MN-major)
             // x I (K-major), exact in fp32 since every product is base x 1 or x 0
             if (ok && s < K) {
-              const uint32_t bslot = Lb % kNBS;
-              if (!mbar_wait_bounded(&ctl->bfull[bslot], (Lb / kNBS) & 1, a.spin, &hdr->abort)) {
-                record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_BASE, cta, s);
-                ok = false;
-                break;
+              uint32_t a_base[kIL];
+              for (int c = 0; c < nil; ++c) {
+                const uint32_t bslot = (Lb + c) % kNBS;
+                if (!mbar_wait_bounded(&ctl->bfull[bslot], ((Lb + c) / kNBS) & 1, a.spin,
+                                       &hdr->abort)) {
+                  record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_BASE, cta, s);
+                  ok = false;
+                  break;
+                }
+                a_base[c] = smem_u32(sBase + (size_t)bslot * N * kCH);
               }
+              if (!ok) break;
               tc_fence_after();
-              const uint32_t a_base = smem_u32(sBase + (size_t)bslot * N * kCH);
               const uint32_t b_base = smem_u32(sI);
 #pragma unroll
               for (int kk = 0; kk < N / 16; ++kk) {
-                const uint64_t ad = smem_desc_sw128(a_base + kk * 2048, N * 128, 1024);
                 const uint64_t bd = smem_desc_sw128(b_base + kk * 32, 16, 1024);
-                umma_bf16(dcol, ad, bd, idesc, 1u);
+#pragma unroll
+                for (int c = 0; c < kIL; ++c) {
+                  if (c >= nil) break;
+                  const uint64_t ad = smem_desc_sw128(a_base[c] + kk * 2048, N * 128, 1024);
+                  umma_bf16(taddr + (uint32_t)((c0 + c) * N), ad, bd, idesc, 1u);
+                }
               }
-              umma_commit(&ctl->bempty[bslot]);
-              ++Lb;
+              for (int c = 0; c < nil; ++c) umma_commit(&ctl->bempty[(Lb + c) % kNBS]);
+              Lb += nil;
             }
-            if (ok) umma_commit(&ctl->dfull[cl]);
-            if (a.trace && cta == 0 && g == 0 && cl < 8)
-              a.trace[(size_t)min(s, K) * kTracePhases + 24 + cl] = globaltimer_ns();
+            if (!ok) break;
+            for (int c = 0; c < nil; ++c) {
+              umma_commit(&ctl->dfull[c0 + c]);
+              if (a.trace && cta == 0 && g == 0 && c0 + c < 8)
+                a.trace[(size_t)min(s, K) * kTracePhases + 24 + c0 + c] = globaltimer_ns();
+            }
           }
           if (a.trace && cta == 0 && g == 0) a.trace[(size_t)min(s, K) * kTracePhases + 10] = globaltimer_ns();
         }
@@ -723,11 +765,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               }
               if (!a.greedy) {
                 if (lm > m[r]) {
-                  s[r] *= exp2f((m[r] - lm) * k);
+                  s[r] *= fexp2((m[r] - lm) * k);
                   m[r] = lm;
                 }
 #pragma unroll
-                for (int j = 0; j < 8; ++j) s[r] += exp2f((e[j] - m[r]) * k);
+                for (int j = 0; j < 8; ++j) s[r] += fexp2((e[j] - m[r]) * k);
               }
             }
         }
@@ -826,76 +868,130 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
     // fin = true: residual / target mass buckets, chosen by ctl->S[n] != 0.
     auto bucket_mass = [&](int n, int cl, int q, bool fin) {
       const float2 p = sBucket[((size_t)cl * 4 + q) * N + n];
-      if (!fin) return p.y > 0.f ? p.y * exp2f((p.x - ctl->M[n]) * k) : 0.f;
+      if (!fin) return p.y > 0.f ? p.y * fexp2((p.x - ctl->M[n]) * k) : 0.f;
       return ctl->S[n] != 0.f ? p.y : p.x;
     };
-    // Bucket walk for every owned row (one warp per row, lanes = buckets),
-    // then per-warp work lists: a row goes to one of the two warps of its
-    // bucket's quadrant.
-    auto walk_and_assign = [&](bool fin) {
+    // Bucket walk for every owned row: warp w walks rows o = w, w + 8, ...
+    // side by side (lanes = buckets, 32 per pass), then loads the logits the
+    // scan of the chosen bucket needs (lanes = its 32 tokens) into tbuf / bbuf:
+    // tgt_row >= 0: that target row (draft steps of a cycle); -1: the stop
+    // row's target and base rows (final step); -2: nothing (drafting only).
+    auto walk_and_assign = [&](bool fin, int g, int tgt_row) {
       const int n_owned = ctl->n_owned;
       const int nbk = ncc * 4;  // buckets in ascending token order
-      for (int o = warp; o < n_owned; o += 8) {
-        const int n = ctl->owned[o];
-        const float tin = ctl->obtarget[o];
-        float carry = 0.f;
-        int pick = -1, lastb = -1;
-        float tin_in = INFINITY;
-        for (int b0 = 0; b0 < nbk && pick < 0; b0 += 32) {  // 32 buckets per pass
+      T tl[kOwnBatch], bl[kOwnBatch];  // logits of the chosen buckets, in flight
+      if (warp < n_owned) {
+        int nn[kOwnBatch], pick[kOwnBatch], lastb[kOwnBatch];
+        float tin[kOwnBatch], carry[kOwnBatch], tin_in[kOwnBatch];
+#pragma unroll
+        for (int j = 0; j < kOwnBatch; ++j) {
+          const int o = warp + 8 * j;
+          const bool has = o < n_owned;
+          nn[j] = ctl->owned[has ? o : warp];
+          tin[j] = has ? ctl->obtarget[o] : 0.f;
+          carry[j] = 0.f;
+          pick[j] = has ? -1 : 0;  // padding slots count as done
+          lastb[j] = -1;
+          tin_in[j] = INFINITY;
+        }
+        for (int b0 = 0; b0 < nbk; b0 += 32) {  // 32 buckets per pass
           const int bk = b0 + lane;
-          const float w = bk < nbk ? bucket_mass(n, bk >> 2, bk & 3, fin) : 0.f;
-          float incl = w;
+          float w[kOwnBatch], incl[kOwnBatch];
+#pragma unroll
+          for (int j = 0; j < kOwnBatch; ++j) {
+            w[j] = bk < nbk ? bucket_mass(nn[j], bk >> 2, bk & 3, fin) : 0.f;
+            incl[j] = w[j];
+          }
 #pragma unroll
           for (int off = 1; off < 32; off <<= 1) {
-            const float y = __shfl_up_sync(FULL, incl, off);
-            if (lane >= off) incl += y;
-          }
-          const unsigned cross = __ballot_sync(FULL, carry + incl > tin);
-          const unsigned pos = __ballot_sync(FULL, w > 0.f);
-          if (pos) lastb = b0 + 31 - __clz(pos);
-          if (cross) {
-            const int l = __ffs(cross) - 1;
-            pick = b0 + l;
-            tin_in = tin - (carry + __shfl_sync(FULL, incl - w, l));
-          }
-          carry += __shfl_sync(FULL, incl, 31);
-        }
-        if (lane == 0) {
-          if (pick < 0) {
-            pick = lastb < 0 ? 0 : lastb;
-            tin_in = INFINITY;
-          }
-          ctl->obucket[o] = pick;
-          ctl->obtarget[o] = tin_in;
-        }
-      }
-      named_sync();
-      // Stage the chosen bucket of every owned row (32 values from tensor
-      // memory, reachable only from the warps of that lane quadrant) into
-      // shared memory, so that any warp can then scan any owned row.
-      {
-        tc_fence_after();
-        int mine = 0;
-        for (int o0 = 0; o0 < n_owned;) {
-          int oo[kOwnBatch];
-          float vv[kOwnBatch];
-          int got = 0;
-          for (; o0 < n_owned && got < kOwnBatch; ++o0) {
-            if ((ctl->obucket[o0] & 3) != q4) continue;
-            if (((mine++) & 1) != (warp >> 2)) continue;
-            oo[got++] = o0;
+#pragma unroll
+            for (int j = 0; j < kOwnBatch; ++j) {
+              const float y = __shfl_up_sync(FULL, incl[j], off);
+              if (lane >= off) incl[j] += y;
+            }
           }
 #pragma unroll
           for (int j = 0; j < kOwnBatch; ++j) {
+            const unsigned cross = __ballot_sync(FULL, carry[j] + incl[j] > tin[j]);
+            const unsigned pos = __ballot_sync(FULL, w[j] > 0.f);
+            const float before = __shfl_sync(FULL, incl[j] - w[j], cross ? __ffs(cross) - 1 : 0);
+            const float total = __shfl_sync(FULL, incl[j], 31);
+            if (pick[j] < 0) {  // uniform across the warp
+              if (pos) lastb[j] = b0 + 31 - __clz(pos);
+              if (cross) {
+                pick[j] = b0 + __ffs(cross) - 1;
+                tin_in[j] = tin[j] - (carry[j] + before);
+              }
+              carry[j] += total;
+            }
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < kOwnBatch; ++j) {
+          if (pick[j] < 0) {
+            pick[j] = lastb[j] < 0 ? 0 : lastb[j];
+            tin_in[j] = INFINITY;
+          }
+          const int o = warp + 8 * j;
+          if (lane == 0 && o < n_owned) {
+            ctl->obucket[o] = pick[j];
+            ctl->obtarget[o] = tin_in[j];
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < kOwnBatch; ++j) {  // issued now, used after the staging below
+          const int n = nn[j];
+          const int64_t b = (int64_t)g * N + n;
+          const int v = min((chunk0 + (pick[j] >> 2)) * kCH + (pick[j] & 3) * 32 + lane, V - 1);
+          const int row = tgt_row >= 0 ? tgt_row : (ctl->alive[n] ? K : ctl->stoprow[n]);
+          if (tgt_row != -2) tl[j] = target[(b * (K + 1) + row) * V + v];
+          if (tgt_row == -1) bl[j] = base[(b * K + min(row, K - 1)) * V + v];
+        }
+      }
+      named_sync();
+      // Stage the chosen bucket of every owned row into shared memory, so that
+      // any warp can scan any owned row.  Tensor memory lanes of a quadrant are
+      // reachable only from its two warps, which take alternate rows.
+      {
+        tc_fence_after();
+        const int h = warp >> 2;
+        const bool m0 = lane < n_owned && (ctl->obucket[lane] & 3) == q4;
+        const bool m1 = lane + 32 < n_owned && (ctl->obucket[lane + 32] & 3) == q4;
+        const unsigned q0 = __ballot_sync(FULL, m0), q1 = __ballot_sync(FULL, m1);
+        const unsigned below = (1u << lane) - 1u;
+        const int r0 = __popc(q0 & below), r1 = __popc(q0) + __popc(q1 & below);
+        const unsigned s0 = __ballot_sync(FULL, m0 && (r0 & 1) == h);
+        const unsigned s1 = __ballot_sync(FULL, m1 && (r1 & 1) == h);
+        unsigned long long rem = ((unsigned long long)s1 << 32) | s0;
+        constexpr int SB = 16;  // rows per batch of tensor-memory loads
+        while (rem) {  // warp-uniform
+          int oo[SB];
+          float vv[SB];
+#pragma unroll
+          for (int j = 0; j < SB; ++j) {
+            oo[j] = rem ? __ffsll((long long)rem) - 1 : -1;
+            rem &= rem - 1;
+          }
+#pragma unroll
+          for (int j = 0; j < SB; ++j) {
             vv[j] = 0.f;
-            if (j >= got) continue;
+            if (oo[j] < 0) continue;
             const int cl = ctl->obucket[oo[j]] >> 2, n = ctl->owned[oo[j]];
             tmem_ld1(taddr + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(cl * N + n), &vv[j]);
           }
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < kOwnBatch; ++j)
-            if (j < got) zbuf[oo[j] * 32 + lane] = vv[j];
+          for (int j = 0; j < SB; ++j)
+            if (oo[j] >= 0) zbuf[oo[j] * 32 + lane] = vv[j];
+        }
+      }
+      if (warp < n_owned) {
+#pragma unroll
+        for (int j = 0; j < kOwnBatch; ++j) {
+          const int o = warp + 8 * j;
+          if (o >= n_owned) continue;
+          if (tgt_row != -2) tbuf[o * 32 + lane] = tl[j];
+          if (tgt_row == -1) bbuf[o * 32 + lane] = bl[j];
         }
       }
       named_sync();
@@ -958,7 +1054,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               }
 #pragma unroll
               for (int t = 0; t < E; ++t)
-                w[t] = (c0 + t < G && v[t].y > 0.f) ? v[t].y * exp2f((v[t].x - M) * k) : 0.f;
+                w[t] = (c0 + t < G && v[t].y > 0.f) ? v[t].y * fexp2((v[t].x - M) * k) : 0.f;
             } else {
               float rt = 0.f, pt = 0.f;
 #pragma unroll
@@ -1045,7 +1141,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             float st = 0.f;
 #pragma unroll
             for (int t = 0; t < E; ++t)
-              if (c0 + t < G && tv[t].y > 0.f) st += tv[t].y * exp2f((tv[t].x - Mt) * k);
+              if (c0 + t < G && tv[t].y > 0.f) st += tv[t].y * fexp2((tv[t].x - Mt) * k);
             rc.Mt = Mt;
             rc.St = warp_sum(st);
           }
@@ -1110,6 +1206,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
         }
         named_sync();
         gather_u(nb_g);
+        if (!a.greedy && a.mode == MODE_CYCLE && tid < nb_g)  // accept-test uniform of the step
+          ctl->uacc[tid] = philox_uniform(a.seed, a.cycle, a.row0 + (uint32_t)(g * N + tid),
+                                          (uint32_t)i, TAG_ACCEPT);
         // pull the next target row of every live batch row into L2 now; the
         // background pass reads it while this step's barrier completes
         if (a.mode == MODE_CYCLE && tid < nb_g && ctl->alive[tid])
@@ -1179,7 +1278,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
 #pragma unroll
               for (int j = 0; j < NCOL; ++j) {
                 rmax[j] = fmaxf(rmax[j], d[j]);
-                d[j] = valid ? exp2f((d[j] - ctl->ref[n0 + j]) * k) : 0.f;
+                d[j] = valid ? fexp2((d[j] - ctl->ref[n0 + j]) * k) : 0.f;
               }
               bfly_sum1<NCOL>(d, lane);
               if ((lane & (REP - 1)) == 0)
@@ -1298,7 +1397,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           if (TC && tid == 0) mbar_arrive(&ctl->tfree);
         } else {
           // ---------------- owners: bucket walk, then batched bucket scans
-          walk_and_assign(false);
+          walk_and_assign(false, g, a.mode == MODE_CYCLE ? i : -2);
           mark(g, i, 15);
           const int n_owned = ctl->n_owned;
           if (warp < n_owned) {  // owned rows o = warp, warp + 8, ... (n_owned <= N <= 64)
@@ -1320,20 +1419,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               const int v = v0 + lane;
               const bool valid = v < V;
               const float z = valid ? dv[j] : -INFINITY;  // z = base + bias, kept in tensor memory
-              const float e = valid ? exp2f((z - M) * k) : 0.f;
+              const float e = valid ? fexp2((z - M) * k) : 0.f;
               const int wl = bucket_scan(e, ctl->obtarget[oo[j]]);
               dtok[j] = v0 + wl;
               zd[j] = __shfl_sync(FULL, z, wl);
-              qd[j] = exp2f((zd[j] - M) * k) / S;
+              qd[j] = fexp2((zd[j] - M) * k) / S;
             }
             const bool cyc = a.mode == MODE_CYCLE;
 #pragma unroll
-            for (int j = 0; j < kOwnBatch; ++j) {
-              const int oj = oo[j] < 0 ? warp : oo[j];  // slot "warp" is owned
-              const int n = ctl->owned[oj];
-              const int dt = oo[j] < 0 ? 0 : min(max(dtok[j], 0), V - 1);
-              td[j] = cyc ? ld_elem(target, ((int64_t)(g * N + n) * (K + 1) + i) * V + dt) : 0.f;
-            }
+            for (int j = 0; j < kOwnBatch; ++j)  // target logit of the drafted token, staged
+              td[j] = (cyc && oo[j] >= 0) ? to_f<T>(tbuf[oo[j] * 32 + (dtok[j] & 31)]) : 0.f;
 #pragma unroll
             for (int j = 0; j < kOwnBatch; ++j) {
               if (oo[j] < 0) continue;
@@ -1345,10 +1440,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               float pd = NaNf;
               if (alive) {
                 const float Mt = ctl->Mt[n], St = ctl->St[n];
-                pd = exp2f((td[j] - Mt) * k) / St;
-                const float ratio = exp2f(((td[j] - Mt) - (zd[j] - M)) * k) * (S / St);
-                const float uacc = philox_uniform(a.seed, a.cycle, a.row0 + (uint32_t)b, (uint32_t)i, TAG_ACCEPT);
-                accept = uacc < fminf(ratio, 1.0f) ? 1 : 0;
+                pd = fexp2((td[j] - Mt) * k) / St;
+                const float ratio = fexp2(((td[j] - Mt) - (zd[j] - M)) * k) * (S / St);
+                accept = ctl->uacc[n] < fminf(ratio, 1.0f) ? 1 : 0;
               }
               if (lane == 0) {
                 a.tokens[((int64_t)par * K + i) * N + n] = dtok[j];
@@ -1488,10 +1582,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               const int n = n0 + j;
               float r = 0.f, p = 0.f;
               if (valid && n < nb_g) {
-                p = exp2f((tv[j] - ctl->fMt[n]) * k) * ctl->rfSt[n];
+                p = fexp2((tv[j] - ctl->fMt[n]) * k) * ctl->rfSt[n];
                 r = p;
                 if (!ctl->alive[n])
-                  r = fmaxf(p - exp2f((d[j] + bvv[j] - ctl->zM[n]) * k) * ctl->rzS[n], 0.f);
+                  r = fmaxf(p - fexp2((d[j] + bvv[j] - ctl->zM[n]) * k) * ctl->rzS[n], 0.f);
               }
               tv[j] = r;
               bvv[j] = p;
@@ -1539,7 +1633,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             }
           }
           named_sync();
-          walk_and_assign(true);
+          walk_and_assign(true, g, -1);
           const int n_owned = ctl->n_owned;
           if (warp < n_owned) {  // owned rows o = warp, warp + 8, ...
             int oo[kOwnBatch];
@@ -1550,14 +1644,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               dv[j] = oo[j] < 0 ? 0.f : zbuf[oo[j] * 32 + lane];
             }
 #pragma unroll
-            for (int j = 0; j < kOwnBatch; ++j) {  // loads from clamped valid addresses
+            for (int j = 0; j < kOwnBatch; ++j) {  // stop rows' logits, staged by the walk
               const int oj = oo[j] < 0 ? warp : oo[j];  // slot "warp" is owned
-              const int bk = ctl->obucket[oj], n = ctl->owned[oj];
-              const int b = g * N + n;
-              const int row = ctl->alive[n] ? K : ctl->stoprow[n];
-              const int v = min((chunk0 + (bk >> 2)) * kCH + (bk & 3) * 32 + lane, V - 1);
-              tvv[j] = ld_elem(target, ((int64_t)b * (K + 1) + row) * V + v);
-              bvv[j] = ld_elem(base, ((int64_t)b * K + min(row, K - 1)) * V + v);
+              tvv[j] = to_f<T>(tbuf[oj * 32 + lane]);
+              bvv[j] = to_f<T>(bbuf[oj * 32 + lane]);
             }
 #pragma unroll
             for (int j = 0; j < kOwnBatch; ++j) {
@@ -1571,10 +1661,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               const int v = v0 + lane;
               float w = 0.f;
               if (v < V) {
-                const float p = exp2f((tvv[j] - ctl->fMt[n]) * k) * ctl->rfSt[n];
+                const float p = fexp2((tvv[j] - ctl->fMt[n]) * k) * ctl->rfSt[n];
                 w = p;
                 if (!bonus && !use_p)
-                  w = fmaxf(p - exp2f((dv[j] + bvv[j] - ctl->zM[n]) * k) * ctl->rzS[n], 0.f);
+                  w = fmaxf(p - fexp2((dv[j] + bvv[j] - ctl->zM[n]) * k) * ctl->rzS[n], 0.f);
               }
               const int wl = bucket_scan(w, ctl->obtarget[oo[j]]);
               if (lane == 0) a.out[(int64_t)b * (K + 1) + row] = v0 + wl;
@@ -1632,7 +1722,8 @@ size_t smem_bytes(int r, int nc) {
   const int nkb = r / 64;
   size_t s = 1024;  // alignment slack
   if (TC) s += (size_t)kNS * kWStage;
-  const size_t u = TC ? (size_t)nkb * N * 128 : (size_t)N * r * 4;
+  const size_t u = u_region_bytes<T, TC, N>(r);
+  (void)nkb;
   s += (u + 1023) & ~size_t(1023);
   if (TC) s += (size_t)N * 128;  // identity operand
   s += (size_t)kNBS * N * kCH * sizeof(T);

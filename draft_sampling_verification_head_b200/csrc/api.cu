@@ -65,12 +65,13 @@ size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
-bool make_tmap_W(CUtensorMap* m, const void* W, int r, int V) {
+// W [r, V] bf16: boxes of 64 tokens x box_k rank rows, 128-byte swizzle.
+bool make_tmap_W(CUtensorMap* m, const void* W, int r, int V, int box_k) {
   EncodeTiledFn f = encode_fn();
   if (!f) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)V, (cuuint64_t)r};
   const cuuint64_t strides[1] = {(cuuint64_t)V * 2};
-  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_k};
   const cuuint32_t estr[2] = {1, 1};
   return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(W), dims, strides, box, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -200,7 +201,7 @@ spec_status spec_markov_bias(const spec_params* p, const void* U, const void* W,
   cudaError_t e;
   if (tc) {
     CUtensorMap tm;
-    if (!make_tmap_W(&tm, W, p->r, p->V)) return SPEC_ERR_CUDA;
+    if (!make_tmap_W(&tm, W, p->r, p->V, 64)) return SPEC_ERR_CUDA;
     e = launch_bias_tc(tm, reinterpret_cast<const __nv_bfloat16*>(U), prev, bias, p->B, p->V,
                        p->r, header_of(ws), spin_of(p), st);
   } else if (p->dtype == SPEC_BF16) {
@@ -239,7 +240,7 @@ static spec_status run_cycle(const spec_params* p, int mode, const void* base, c
   }
   CUtensorMap tmW, tmBase;
   memset(&tmW, 0, sizeof(tmW));
-  if (g.tc && !make_tmap_W(&tmW, W, p->r, p->V)) return SPEC_ERR_CUDA;
+  if (g.tc && !make_tmap_W(&tmW, W, p->r, p->V, kCycleWBoxK)) return SPEC_ERR_CUDA;
   if (!make_tmap_base(&tmBase, base, p->dtype, p->B, p->K, p->V, g.N, g.tc)) return SPEC_ERR_CUDA;
   CycleLaunch L;
   L.base = base;

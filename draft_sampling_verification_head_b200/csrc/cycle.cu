@@ -52,7 +52,12 @@ constexpr int kNS = 6;              // W ring stages
 constexpr int kNBS = 4;             // base tile ring stages
 constexpr int kIL = 1;              // chunks whose MMA chains are interleaved
 constexpr int kMaxNC = 32;
-constexpr int kWStage = kCH * 64 * 2;  // 16 KB: 128 tokens x 64 rank, bf16
+// One W ring stage = kKS MMA K-steps (16 rank rows each) of up to kIL
+// chunks: per chunk and K-step two 64-token halves of [16 rows][128 B],
+// 128-byte swizzled.
+constexpr int kKS = 4 / kIL;                     // K-steps per stage
+constexpr int kWChunk = kCH * 16 * 2;            // 4 KB per chunk and K-step
+constexpr int kWStage = kIL * kKS * kWChunk;     // 16 KB
 constexpr int kMaxG = 160;          // CTAs a launch may use (>= SM count); partial-row stride
 constexpr int kOwnBatch = 8;        // owned rows scanned together by one warp
 constexpr unsigned FULL = 0xffffffffu;
@@ -445,27 +450,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
       bool ok = true;
       for (int g = 0; g < a.ngroups && ok; ++g) {
         for (int s = 0; s < nsteps && ok; ++s) {
-          // stages in the MMA's order: k-block by k-block over kIL chunks at a time
+          // stages in the MMA's order: K-step by K-step over kIL chunks at a time
           for (int c0 = 0; c0 < ncc && ok; c0 += kIL) {
             const int nil = min(kIL, ncc - c0);
-            for (int kb = 0; kb < nkb && ok; ++kb) {
-              for (int c = 0; c < nil; ++c) {
-                const int v0 = (chunk0 + c0 + c) * kCH;
-                const uint32_t slot = Lw % kNS;
-                if (Lw >= kNS &&
-                    !mbar_wait_bounded(&ctl->wempty[slot], ((Lw / kNS) - 1) & 1, a.spin,
-                                       &hdr->abort)) {
-                  record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_FULL, cta, 100 + s);
-                  ok = false;
-                  break;
-                }
-                mbar_arrive_expect_tx(&ctl->wfull[slot], kWStage);
-                tma_load_2d(sW + (size_t)slot * kWStage, &a.tmW, &ctl->wfull[slot], v0, kb * 64,
-                            polW);
-                tma_load_2d(sW + (size_t)slot * kWStage + kWStage / 2, &a.tmW,
-                            &ctl->wfull[slot], v0 + 64, kb * 64, polW);
-                ++Lw;
+            for (int ks0 = 0; ks0 < nkb * 4; ks0 += kKS) {
+              const uint32_t slot = Lw % kNS;
+              if (Lw >= kNS &&
+                  !mbar_wait_bounded(&ctl->wempty[slot], ((Lw / kNS) - 1) & 1, a.spin,
+                                     &hdr->abort)) {
+                record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_FULL, cta, 100 + s);
+                ok = false;
+                break;
               }
+              mbar_arrive_expect_tx(&ctl->wfull[slot], (uint32_t)(nil * kKS * kWChunk));
+              for (int j = 0; j < kKS; ++j)
+                for (int c = 0; c < nil; ++c) {
+                  const int v0 = (chunk0 + c0 + c) * kCH;
+                  uint8_t* dst = sW + (size_t)slot * kWStage + (size_t)(j * kIL + c) * kWChunk;
+                  tma_load_2d(dst, &a.tmW, &ctl->wfull[slot], v0, (ks0 + j) * 16, polW);
+                  tma_load_2d(dst + kWChunk / 2, &a.tmW, &ctl->wfull[slot], v0 + 64,
+                              (ks0 + j) * 16, polW);
+                }
+              ++Lw;
             }
           }
         }
@@ -579,37 +585,35 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           tc_fence_after();
           if (a.trace && cta == 0 && g == 0) a.trace[(size_t)min(s, K) * kTracePhases + 9] = globaltimer_ns();
           // kIL chunks at a time, their MMAs alternating: each chunk's K-steps
-          // accumulate into its own columns, so the chains overlap in the pipe
+          // accumulate into its own columns, so consecutive MMAs are independent
           for (int c0 = 0; c0 < ncc && ok; c0 += kIL) {
             const int nil = min(kIL, ncc - c0);
-            for (int kb = 0; kb < nkb && ok; ++kb) {
-              uint32_t a_base[kIL];
-              for (int c = 0; c < nil; ++c) {
-                const uint32_t slot = (Lw + c) % kNS;
-                if (!mbar_wait_bounded(&ctl->wfull[slot], ((Lw + c) / kNS) & 1, a.spin,
-                                       &hdr->abort)) {
-                  record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_FULL, cta, s);
-                  ok = false;
-                  break;
-                }
-                a_base[c] = smem_u32(sW + (size_t)slot * kWStage);
+            for (int ks0 = 0; ks0 < nkb * 4; ks0 += kKS) {
+              const uint32_t slot = Lw % kNS;
+              if (!mbar_wait_bounded(&ctl->wfull[slot], (Lw / kNS) & 1, a.spin, &hdr->abort)) {
+                record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_FULL, cta, s);
+                ok = false;
+                break;
               }
-              if (!ok) break;
               tc_fence_after();
-              const uint32_t b_base = smem_u32(sU + (size_t)kb * N * 128);
+              const uint32_t a_base = smem_u32(sW + (size_t)slot * kWStage);
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t bd = smem_desc_sw128(b_base + kk * 32, 16, 1024);
+              for (int j = 0; j < kKS; ++j) {
+                const int ks = ks0 + j;
+                const uint64_t bd = smem_desc_sw128(
+                    smem_u32(sU + (size_t)(ks >> 2) * N * 128) + (ks & 3) * 32, 16, 1024);
 #pragma unroll
                 for (int c = 0; c < kIL; ++c) {
                   if (c >= nil) break;
-                  const uint64_t ad = smem_desc_sw128(a_base[c] + kk * 2048, 8192, 1024);
-                  umma_bf16(taddr + (uint32_t)((c0 + c) * N), ad, bd, idesc, (kb | kk) != 0);
+                  const uint64_t ad =
+                      smem_desc_sw128(a_base + (j * kIL + c) * kWChunk, kWChunk / 2, 1024);
+                  umma_bf16(taddr + (uint32_t)((c0 + c) * N), ad, bd, idesc, ks != 0);
                 }
               }
-              for (int c = 0; c < nil; ++c) umma_commit(&ctl->wempty[(Lw + c) % kNS]);
-              Lw += nil;
+              umma_commit(&ctl->wempty[slot]);
+              ++Lw;
             }
+            if (!ok) break;
             // z = bias + base: D += base^T (M = tokens, K = batch rows, MN-major)
             // x I (K-major), exact in fp32 since every product is base x 1 or x 0
             if (ok && s < K) {

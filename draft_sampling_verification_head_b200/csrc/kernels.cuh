@@ -81,7 +81,8 @@ cudaError_t launch_cycle(const CycleLaunch& L, const CycleGeom& g, WsHeader* hdr
                          const CUtensorMap* tmW, const CUtensorMap* tmBase, cudaStream_t st);
 
 // ---- Tensor maps --------------------------------------------------------------
-bool make_tmap_W(CUtensorMap* m, const void* W, int r, int V);
+bool make_tmap_W(CUtensorMap* m, const void* W, int r, int V, int box_k);
+constexpr int kCycleWBoxK = 16;  // rank rows per W box of the fused cycle (one MMA K-step)
 bool make_tmap_base(CUtensorMap* m, const void* base, int dtype, int B, int K, int V, int N,
                     bool tc);
 

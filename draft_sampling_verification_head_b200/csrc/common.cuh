@@ -213,6 +213,18 @@ SPEC_DEV void tma_load_2d(void* dst, const CUtensorMap* m, uint64_t* bar, int32_
       "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
+// 16-byte asynchronous copy global -> shared (bypassing L1), grouped by
+// commit_group / wait_group.  Both addresses 16-byte aligned.
+SPEC_DEV void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+SPEC_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int PENDING>
+SPEC_DEV void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(PENDING) : "memory");
+}
+
 // Untiled bulk copy global -> this CTA's shared memory, completion counted in
 // bytes on the mbarrier.  Both addresses 16-byte aligned, bytes a multiple of 16.
 SPEC_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar,

@@ -92,8 +92,8 @@ struct Args {
 template <int N>
 struct Ctl {
   uint64_t wfull[kNS], wempty[kNS], bfull[kNBS], bempty[kNBS], dfull[kMaxNC];
-  uint64_t ffull[kNBS], fempty[kNBS];  // final step: gathered stop-row tiles in the base ring
-  uint64_t bready, tfree, mmadone, rows_known;
+  uint64_t bready, tfree, mmadone;
+  uint64_t ring_free;  // the final step no longer needs the base ring slots
   uint32_t tmem_slot;
   int32_t abort_local;
   int32_t n_owned;
@@ -108,10 +108,11 @@ struct Ctl {
   float zM[N], zS[N];   // draft stats of the stop row
   float Mt[N], St[N];   // target stats of row i during a step
   float fMt[N], fSt[N]; // target stats of the final row (stop row or row K)
-  float rfSt[N], rzS[N]; // 1 / fSt and 1 / zS for the final step
   float uacc[N];        // accept-test uniform of the current step
-  float ref[N];         // per-row reference of the fast path (previous step's max)
+  alignas(16) float ref[N];  // per-row reference of the fast path (previous step's max)
   float cmax[4][N];     // true max per row and tensor-memory quadrant
+  float psum[4][N];     // fast path: this CTA's sum per row and tensor-memory quadrant
+  alignas(16) float4 fcst[N];  // final step per row: target max, 1 / target sum, draft max, 1 / draft sum
   int32_t redo;
 };
 
@@ -408,12 +409,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
       mbar_init(&ctl->bfull[i], 1);
       mbar_init(&ctl->bempty[i], TC ? 1 : kComputeThreads / 32);  // TC: freed by the MMA
     }
-    for (int i = 0; i < kNBS; ++i) {
-      mbar_init(&ctl->ffull[i], 1);
-      mbar_init(&ctl->fempty[i], kComputeThreads / 32);
-    }
     for (int i = 0; i < kMaxNC; ++i) mbar_init(&ctl->dfull[i], 1);
-    mbar_init(&ctl->rows_known, 1);
+    mbar_init(&ctl->ring_free, 1);
     mbar_init(&ctl->bready, 1);
     mbar_init(&ctl->tfree, 1);
     mbar_init(&ctl->mmadone, 1);
@@ -482,13 +479,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
     }
   } else if (warp == kBaseWarp) {
     // Draft steps: one base tile [N rows x 128 tokens] per chunk and step, by
-    // lane 0 through the tensor map.  Final step (stochastic cycle): for each
-    // chunk a target tile and a base tile of the rows' stop rows (row K for a
-    // row that accepted every draft), gathered row by row with bulk copies by
-    // all 32 lanes once the stop rows are known.
+    // lane 0 through the tensor map.  (The final step's stop-row tiles are
+    // gathered into the same slots by the compute warps.)
     const uint64_t polB = policy_evict_first();
     if (lane == 0) tma_prefetch_desc(&a.tmBase);
-    uint32_t Lb = 0, Lf = 0;
+    uint32_t Lb = 0;
     int ok = 1;
     auto wait0 = [&](uint64_t* bar, uint32_t parity, int where) {  // lane 0 waits, all learn
       int r = 1;
@@ -499,9 +494,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
       return __shfl_sync(FULL, r, 0);
     };
     for (int g = 0; g < a.ngroups && ok; ++g) {
-      // slots last held final-step tiles of the previous group: wait until read
-      for (uint32_t L = (Lf > kNBS ? Lf - kNBS : 0); L < Lf && ok; ++L)
-        ok = wait0(&ctl->fempty[L % kNBS], (L / kNBS) & 1, 2000 + g);
+      // the previous group's final step gathers its stop rows into these
+      // slots: start this group's tiles once it has finished with them
+      if (g > 0 && has_final) ok = wait0(&ctl->ring_free, (uint32_t)(g - 1) & 1, 2000 + g);
       for (int s = 0; s < K && ok; ++s) {
         for (int cl = 0; cl < ncc && ok; ++cl) {
           const uint32_t slot = Lb % kNBS;
@@ -522,43 +517,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           ++Lb;
         }
       }
-      if (!has_final || !ok) continue;
-      // every draft tile read, stop rows of this group known
-      for (uint32_t L = (Lb > kNBS ? Lb - kNBS : 0); L < Lb && ok; ++L)
-        ok = wait0(&ctl->bempty[L % kNBS], (L / kNBS) & 1, 1000 + g);
-      if (ok) ok = wait0(&ctl->rows_known, (uint32_t)g & 1, 3000 + g);
-      const int nb_g = min(N, a.B - g * N);
-      for (int cl = 0; cl < ncc && ok; ++cl) {
-        const int v0 = (chunk0 + cl) * kCH;
-        const uint32_t bytes = (uint32_t)(min(kCH, V - v0) * sizeof(T));
-        for (int t = 0; t < 2 && ok; ++t) {  // t = 0: target rows, t = 1: base rows
-          const uint32_t slot = Lf % kNBS;
-          if (Lf >= kNBS) ok = wait0(&ctl->fempty[slot], ((Lf / kNBS) - 1) & 1, 4000 + cl);
-          if (!ok) break;
-          int rows = 0;
-          for (int n = 0; n < nb_g; ++n) rows += (t == 0 || !ctl->alive[n]) ? 1 : 0;
-          if (lane == 0) mbar_arrive_expect_tx(&ctl->ffull[slot], (uint32_t)rows * bytes);
-          __syncwarp();
-          T* dst = sBase + (size_t)slot * N * kCH;
-          for (int n = lane; n < nb_g; n += 32) {
-            const bool alive = ctl->alive[n] != 0;
-            if (t == 1 && alive) continue;
-            const int row = alive ? K : ctl->stoprow[n];
-            const int64_t b = (int64_t)g * N + n;
-            const T* src = t == 0 ? target + (b * (K + 1) + row) * V + v0
-                                  : base + (b * K + row) * V + v0;
-            bulk_load(dst + (size_t)n * kCH, src, bytes, &ctl->ffull[slot], polB);
-          }
-          ++Lf;
-        }
-      }
     }
     // nothing in flight at exit: the latest copy into every slot has landed
     if (lane == 0) {
       for (uint32_t L = (Lb > kNBS ? Lb - kNBS : 0); L < Lb; ++L)
         mbar_drain(&ctl->bfull[L % kNBS], (L / kNBS) & 1);
-      for (uint32_t L = (Lf > kNBS ? Lf - kNBS : 0); L < Lf; ++L)
-        mbar_drain(&ctl->ffull[L % kNBS], (L / kNBS) & 1);
     }
   }
   // =========================================================================
@@ -664,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
   else {
     const int q4 = warp & 3;         // tensor-memory lane quadrant
     const int n0 = (warp >> 2) * NCOL;  // first column (batch row) of this warp
-    uint32_t step_ctr = 0, Lb = 0, Lf = 0;
+    uint32_t step_ctr = 0, Lb = 0;
     uint32_t nbar = 0, tok_expected = 0, rec_expected = 0;
     // Failures are folded into the CTA-wide flag ctl->abort_local; it is only
     // read right after a named barrier, so every compute thread takes the same
@@ -866,6 +829,32 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
       if (cross) return __ffs(cross) - 1;
       const unsigned pos = __ballot_sync(FULL, wv > 0.f);
       return pos ? 31 - __clz(pos) : 0;
+    };
+
+    // Final step: chunk cl's target tile (every row's stop row, or row K) and
+    // base tile (rows that stopped) into base-ring slots 2(cl&1), 2(cl&1)+1,
+    // as 16-byte asynchronous copies by all compute threads, one commit group
+    // per chunk.  Rows past the batch, stopped rows' base and tokens past V are
+    // left stale and only read under guards.
+    auto final_tiles_issue = [&](int g, int cl, int nb_g) {
+      constexpr int EPP = 16 / (int)sizeof(T);  // elements per 16-byte piece
+      constexpr int PPR = kCH / EPP;            // pieces per 128-token row
+      T* tt = sBase + (size_t)((cl & 1) * 2) * N * kCH;
+      T* bt = tt + (size_t)N * kCH;
+      const int v0 = (chunk0 + cl) * kCH;
+      const int npc = min(kCH, V - v0) / EPP;
+      for (int idx = tid; idx < 2 * N * PPR; idx += kComputeThreads) {
+        const int t = idx / (N * PPR), n = (idx / PPR) % N, pc = idx % PPR;
+        if (n >= nb_g || pc >= npc) continue;
+        const bool alive = ctl->alive[n] != 0;
+        if (t == 1 && alive) continue;
+        const int row = alive ? K : ctl->stoprow[n];
+        const int64_t b = (int64_t)g * N + n;
+        const T* src = t == 0 ? target + (b * (K + 1) + row) * V + v0 + pc * EPP
+                              : base + (b * K + row) * V + v0 + pc * EPP;
+        cp_async16((t == 0 ? tt : bt) + (size_t)n * kCH + pc * EPP, src);
+      }
+      cp_async_commit();
     };
 
     // fin = false: softmax buckets (m, s) in the scale of ctl->M[n];
@@ -1226,6 +1215,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
         for (int attempt = 0; attempt < 2; ++attempt) {
           // ---------------- epilogue: z = base + bias, bucket statistics
           uint64_t t_wait = 0, t_base = 0, t_st = 0;
+          float psum = 0.f;
           float rmax[NCOL];
 #pragma unroll
           for (int j = 0; j < NCOL; ++j) rmax[j] = -INFINITY;
@@ -1279,12 +1269,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               bfly_amax<NCOL>(d, ix, lane);
               if ((lane & (REP - 1)) == 0) bk[n0 + lane / REP] = make_float2(d[0], __int_as_float(ix[0]));
             } else if (fast) {
+              const float4* r4 = reinterpret_cast<const float4*>(ctl->ref + n0);
 #pragma unroll
-              for (int j = 0; j < NCOL; ++j) {
-                rmax[j] = fmaxf(rmax[j], d[j]);
-                d[j] = valid ? fexp2((d[j] - ctl->ref[n0 + j]) * k) : 0.f;
+              for (int j4 = 0; j4 < NCOL / 4; ++j4) {
+                const float4 rr = r4[j4];
+                const float rv[4] = {rr.x, rr.y, rr.z, rr.w};
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                  const int j = 4 * j4 + t;
+                  rmax[j] = fmaxf(rmax[j], d[j]);
+                  d[j] = valid ? fexp2((d[j] - rv[t]) * k) : 0.f;
+                }
               }
               bfly_sum1<NCOL>(d, lane);
+              psum += d[0];  // this lane's column, summed over the CTA's chunks
               if ((lane & (REP - 1)) == 0)
                 bk[n0 + lane / REP] = make_float2(ctl->ref[n0 + lane / REP], d[0]);
             } else {
@@ -1297,9 +1295,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             if (trace && g == 0 && cl < 8 && attempt == 0)
               trace[(size_t)i * kTracePhases + 16 + cl] = globaltimer_ns();
           }
-          if (fast) {  // true max of z per row over this warp's tokens
+          if (fast) {  // true max of z per row over this warp's tokens, and its sum
             bfly_max1<NCOL>(rmax, lane);
-            if ((lane & (32 / NCOL - 1)) == 0) ctl->cmax[q4][n0 + lane / (32 / NCOL)] = rmax[0];
+            if ((lane & (32 / NCOL - 1)) == 0) {
+              ctl->cmax[q4][n0 + lane / (32 / NCOL)] = rmax[0];
+              ctl->psum[q4][n0 + lane / (32 / NCOL)] = psum;
+            }
           }
           tc_fence_before();  // z stores above are read by other warps after the barrier
           named_sync();
@@ -1310,8 +1311,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             trace[(size_t)i * kTracePhases + 13] = t_base;
             trace[(size_t)i * kTracePhases + 14] = t_st;
           }
-          // ---------------- CTA partial per batch row (TPB threads per row)
-          {
+          // ---------------- CTA partial per batch row
+          if (fast) {  // common reference: the four quadrants' running sums
+            if (tid < N) {
+              const int n = tid;
+              const float sum = (ctl->psum[0][n] + ctl->psum[1][n]) + (ctl->psum[2][n] + ctl->psum[3][n]);
+              const float tmax = fmaxf(fmaxf(ctl->cmax[0][n], ctl->cmax[1][n]),
+                                       fmaxf(ctl->cmax[2][n], ctl->cmax[3][n]));
+              a.dpart[(((int64_t)par * (K + 1) + i) * N + n) * kMaxG + cta] =
+                  make_float4(ctl->ref[n], sum, tmax, 0.f);
+            }
+          } else {  // (max, sum) pairs or arg-max over the buckets, TPB threads per row
             const int n = grp_n;
             float m = -INFINITY, s = 0.f;
             int32_t ai = 0x7fffffff;
@@ -1331,14 +1341,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               else
                 ms_combine(m, s, m2, s2, k);
             }
-            if (grp_sub == 0) {
-              float tmax = m;
-              if (fast)
-                tmax = fmaxf(fmaxf(ctl->cmax[0][n], ctl->cmax[1][n]),
-                             fmaxf(ctl->cmax[2][n], ctl->cmax[3][n]));
+            if (grp_sub == 0)
               a.dpart[(((int64_t)par * (K + 1) + i) * N + n) * kMaxG + cta] =
-                  a.greedy ? make_float4(m, __int_as_float(ai), m, 0.f) : make_float4(m, s, tmax, 0.f);
-            }
+                  a.greedy ? make_float4(m, __int_as_float(ai), m, 0.f) : make_float4(m, s, m, 0.f);
           }
           grid_arrive();
           mark(g, i, 3);
@@ -1484,9 +1489,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             ctl->tok[n] = __ldcg(a.tokens + ((int64_t)par * K + i) * N + n);
             if (a.mode == MODE_CYCLE && ctl->alive[n] &&
                 !__ldcg(a.accf + ((int64_t)par * K + i) * N + n)) {
-              const uint32_t sl = (uint32_t)((vslice_hi - vslice_lo) * sizeof(T));
-              prefetch_l2_bulk(target + ((int64_t)(g * N + n) * (K + 1) + i) * V + vslice_lo, sl);
-              prefetch_l2_bulk(base + ((int64_t)(g * N + n) * K + i) * V + vslice_lo, sl);
               ctl->alive[n] = 0;
               ctl->stoprow[n] = i;
               ctl->zM[n] = ctl->M[n];  // draft statistics of the stop row
@@ -1504,8 +1506,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
         }
       }  // draft steps
       if (failed) break;
-      // alive / stoprow are final: the producer may gather the stop rows
-      if (has_final && tid == 0) mbar_arrive(&ctl->rows_known);
+      // alive / stoprow are final: pull this CTA's slice of each row's final
+      // target row (and stop-row base row) into L2, and start copying the first
+      // two chunks' tiles, while the final step's first exchange runs.  The
+      // base ring is idle here: every draft tile of the group has been read,
+      // and the base producer waits for ring_free before the next group.
+      if (has_final) {
+        if (tid < nb_g) {
+          const bool alive = ctl->alive[tid] != 0;
+          const int row = alive ? K : ctl->stoprow[tid];
+          const uint32_t sl = (uint32_t)((vslice_hi - vslice_lo) * sizeof(T));
+          prefetch_l2_bulk(target + ((int64_t)(g * N + tid) * (K + 1) + row) * V + vslice_lo, sl);
+          if (!alive) prefetch_l2_bulk(base + ((int64_t)(g * N + tid) * K + row) * V + vslice_lo, sl);
+        }
+        final_tiles_issue(g, 0, nb_g);
+        if (ncc > 1) final_tiles_issue(g, 1, nb_g);
+      }
 
       if (a.mode == MODE_CYCLE) {
         // row-K target partials (written after the last barrier) become visible
@@ -1544,59 +1560,64 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               if (p < 0 || p >= V) p = 0;
             }
             ctl->prev[n] = p;
-            if (n < nb_g) {
-              ctl->rfSt[n] = 1.f / ctl->fSt[n];
-              ctl->rzS[n] = ctl->alive[n] ? 0.f : 1.f / ctl->zS[n];
-            }
+            if (n < nb_g)  // final-row constants, read once per column and chunk
+              ctl->fcst[n] = make_float4(ctl->fMt[n], 1.f / ctl->fSt[n], ctl->zM[n],
+                                         ctl->alive[n] ? 0.f : 1.f / ctl->zS[n]);
           }
           named_sync();
           gather_u(nb_g);
           mark(g, K, 2);
+          uint64_t t_fmma = 0, t_ftile = 0;
           for (int cl = 0; cl < ncc; ++cl) {
             float d[NCOL];
+            const uint64_t t_m0 = trace ? globaltimer_ns() : 0;
             bias_tile(cl, d);
+            if (trace) t_fmma += globaltimer_ns() - t_m0;
             const int v = (chunk0 + cl) * kCH + q4 * 32 + lane;
             const bool valid = v < V;
-            // gathered stop-row tiles (entries past the copied rows / tokens are
-            // stale and only read under the guards below)
+            // gathered stop-row tiles of this chunk (entries past the copied
+            // rows / tokens are stale and only read under the guards below)
             float tv[NCOL], bvv[NCOL];
             {
-              const uint32_t ts = Lf % kNBS, bs = (Lf + 1) % kNBS;
-              if (!mbar_wait_bounded(&ctl->ffull[ts], (Lf / kNBS) & 1, a.spin, &hdr->abort) ||
-                  !mbar_wait_bounded(&ctl->ffull[bs], ((Lf + 1) / kNBS) & 1, a.spin, &hdr->abort))
-                soft_fail(SPEC_ERR_TIMEOUT, SITE_MBAR_BASE, cta, 5000 + cl);
-              const T* tt = sBase + (size_t)ts * N * kCH;
-              const T* bt = sBase + (size_t)bs * N * kCH;
+              const uint64_t t_t0 = trace ? globaltimer_ns() : 0;
+              if (cl + 1 < ncc)
+                cp_async_wait<1>();  // this thread's copies of chunk cl have landed
+              else
+                cp_async_wait<0>();
+              named_sync();          // ... and every other thread's
+              if (trace) t_ftile += globaltimer_ns() - t_t0;
+              const T* tt = sBase + (size_t)((cl & 1) * 2) * N * kCH;
+              const T* bt = tt + (size_t)N * kCH;
               const int vl = q4 * 32 + lane;
 #pragma unroll
               for (int j = 0; j < NCOL; ++j) {
                 tv[j] = to_f<T>(tt[(n0 + j) * kCH + vl]);
                 bvv[j] = to_f<T>(bt[(n0 + j) * kCH + vl]);
               }
-              __syncwarp();
-              if (lane == 0) {
-                mbar_arrive(&ctl->fempty[ts]);
-                mbar_arrive(&ctl->fempty[bs]);
-              }
-              Lf += 2;
+              named_sync();  // slots of chunk cl read by everyone: refill them
+              if (cl + 2 < ncc) final_tiles_issue(g, cl + 2, nb_g);
             }
-            // residual mass r (into tv) and target mass p (into bvv), in place
+            // residual mass r (into tv) and target mass p (into bvv), in place;
+            // a row that accepted everything has 1 / draft sum = 0: r = p
 #pragma unroll
             for (int j = 0; j < NCOL; ++j) {
               const int n = n0 + j;
-              float r = 0.f, p = 0.f;
-              if (valid && n < nb_g) {
-                p = fexp2((tv[j] - ctl->fMt[n]) * k) * ctl->rfSt[n];
-                r = p;
-                if (!ctl->alive[n])
-                  r = fmaxf(p - fexp2((d[j] + bvv[j] - ctl->zM[n]) * k) * ctl->rzS[n], 0.f);
-              }
-              tv[j] = r;
-              bvv[j] = p;
+              const float4 c = ctl->fcst[n];
+              const bool ok = valid && n < nb_g;
+              const float p = fexp2((tv[j] - c.x) * k) * c.y;
+              const float q = c.w != 0.f ? fexp2((d[j] + bvv[j] - c.z) * k) * c.w : 0.f;
+              tv[j] = ok ? fmaxf(p - q, 0.f) : 0.f;
+              bvv[j] = ok ? p : 0.f;
             }
             bfly_sum2<NCOL>(tv, bvv, lane);
             float2* bk = sBucket + ((size_t)cl * 4 + q4) * N;
             if ((lane & (32 / NCOL - 1)) == 0) bk[n0 + lane / (32 / NCOL)] = make_float2(tv[0], bvv[0]);
+            if (trace && g == 0 && cl < 8) trace[(size_t)K * kTracePhases + 16 + cl] = globaltimer_ns();
+          }
+          if (tid == 0) mbar_arrive(&ctl->ring_free);  // last tile read: slots free
+          if (trace && g == 0) {
+            trace[(size_t)K * kTracePhases + 11] = t_fmma;
+            trace[(size_t)K * kTracePhases + 12] = t_ftile;
           }
           named_sync();
           {
@@ -1664,11 +1685,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               const int row = bonus ? K : ctl->stoprow[n];
               const int v = v0 + lane;
               float w = 0.f;
-              if (v < V) {
-                const float p = fexp2((tvv[j] - ctl->fMt[n]) * k) * ctl->rfSt[n];
-                w = p;
-                if (!bonus && !use_p)
-                  w = fmaxf(p - fexp2((dv[j] + bvv[j] - ctl->zM[n]) * k) * ctl->rzS[n], 0.f);
+              if (v < V) {  // the same expressions as the final epilogue's bucket masses
+                const float4 c = ctl->fcst[n];
+                const float p = fexp2((tvv[j] - c.x) * k) * c.y;
+                const float q = c.w != 0.f ? fexp2((dv[j] + bvv[j] - c.z) * k) * c.w : 0.f;
+                w = (bonus || use_p) ? p : fmaxf(p - q, 0.f);
               }
               const int wl = bucket_scan(w, ctl->obtarget[oo[j]]);
               if (lane == 0) a.out[(int64_t)b * (K + 1) + row] = v0 + wl;
@@ -1693,6 +1714,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
         mark(g, K, 6);
       }
     }  // groups
+    cp_async_wait<0>();  // no copy into shared memory outlives the CTA (failure paths)
     (void)soft_fail;
   }
 

@@ -59,7 +59,6 @@ constexpr int kKS = 4 / kIL;                     // K-steps per stage
 constexpr int kWChunk = kCH * 16 * 2;            // 4 KB per chunk and K-step
 constexpr int kWStage = kIL * kKS * kWChunk;     // 16 KB
 constexpr int kMaxG = 160;          // CTAs a launch may use (>= SM count); partial-row stride
-constexpr int kOwnBatch = 8;        // owned rows scanned together by one warp
 constexpr unsigned FULL = 0xffffffffu;
 
 struct Args {
@@ -80,40 +79,14 @@ struct Args {
   float4* dpart;     // [2][K+1][N][kMaxG]: (m, s, true max, 0) or (max, idx, max, 0)
   float2* tpart;     // [2][K+1][N][kMaxG]: (m, s) or (max, idx)
   int32_t* tokens;   // [2][K][N]
-  int32_t* accf;     // [2][K][N]
   struct Rec* rec;   // [2][K+2][N] row records
+  float2* gbk;       // [G][nbk][N] this step's bucket statistics of every CTA
   uint64_t* trace;   // [K+2][kTracePhases] device timeline of CTA 0, or null
   int B, K, V, r, G, nc, nchunks, mode, greedy, ngroups;
   float k;           // log2(e) / T (1 in greedy mode)
   uint64_t seed, cycle, spin;
   uint32_t row0;  // global index of batch row 0 (Philox counter word 1)
-};
-
-template <int N>
-struct Ctl {
-  uint64_t wfull[kNS], wempty[kNS], bfull[kNBS], bempty[kNBS], dfull[kMaxNC];
-  uint64_t bready, tfree, mmadone;
-  uint64_t ring_free;  // the final step no longer needs the base ring slots
-  uint32_t tmem_slot;
-  int32_t abort_local;
-  int32_t n_owned;
-  int32_t owned[N];
-  int32_t obucket[N];
-  float obtarget[N];
-  int32_t prev[N];
-  int32_t alive[N];
-  int32_t stoprow[N];
-  int32_t tok[N];
-  float M[N], S[N];     // global draft stats of the current step
-  float zM[N], zS[N];   // draft stats of the stop row
-  float Mt[N], St[N];   // target stats of row i during a step
-  float fMt[N], fSt[N]; // target stats of the final row (stop row or row K)
-  float uacc[N];        // accept-test uniform of the current step
-  alignas(16) float ref[N];  // per-row reference of the fast path (previous step's max)
-  float cmax[4][N];     // true max per row and tensor-memory quadrant
-  float psum[4][N];     // fast path: this CTA's sum per row and tensor-memory quadrant
-  alignas(16) float4 fcst[N];  // final step per row: target max, 1 / target sum, draft max, 1 / draft sum
-  int32_t redo;
+  int nbk;        // buckets per CTA (4 per chunk)
 };
 
 // One record per batch row and reduction, written by the row's reducer.
@@ -123,13 +96,41 @@ struct alignas(16) Rec {
   float Mt, St;     // target row statistics
   float trem;       // inverse-CDF target inside the owner CTA's slice (inf: last mass)
   int32_t owner;    // CTA that owns the draw
-  int32_t token;    // greedy: arg-max draft token
-  int32_t acc;      // greedy: accept outcome
+  int32_t token;    // draft token of the step (drawn, or the arg-max)
+  int32_t acc;      // accept outcome
   int32_t flags;    // bit 0: redo the step exactly; bit 1: final draw uses p
   int32_t tam;      // greedy: target arg-max
   int32_t pad;
 };
 static_assert(sizeof(Rec) == 48, "records are three 16-byte words");
+
+template <int N>
+struct Ctl {
+  uint64_t wfull[kNS], wempty[kNS], bfull[kNBS], bempty[kNBS], dfull[kMaxNC];
+  uint64_t bready, tfree, mmadone;
+  uint64_t ring_free;  // the final step no longer needs the base ring slots
+  uint32_t tmem_slot;
+  int32_t abort_local;
+  int32_t prev[N];
+  int32_t alive[N];
+  int32_t stoprow[N];
+  int32_t tok[N];
+  float M[N], S[N];     // global draft stats of the current step
+  float zM[N], zS[N];   // draft stats of the stop row
+  float Mt[N], St[N];   // target stats of row i during a step
+  float fMt[N], fSt[N]; // target stats of the final row (stop row or row K)
+  alignas(16) float ref[N];  // per-row reference of the fast path (previous step's max)
+  float cmax[4][N];     // true max per row and tensor-memory quadrant
+  float psum[4][N];     // fast path: this CTA's sum per row and tensor-memory quadrant
+  alignas(16) float4 fcst[N];  // final step per row: target max, 1 / target sum, draft max, 1 / draft sum
+  int32_t redo;
+  Rec rrec[N];          // records of the rows this CTA reduces, before publication
+  float zpart[8][32];   // per-warp partial Markov biases of a draw's 32 tokens
+  int32_t dbk;          // the draw's bucket inside the owner CTA
+  float dtin;           // inverse-CDF target inside that bucket
+};
+
+
 
 SPEC_DEV void store_rec(Rec* dst, const Rec& r) {
   const float4* s4 = reinterpret_cast<const float4*>(&r);
@@ -367,17 +368,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
   uint8_t* sU = sW + (TC ? (size_t)kNS * kWStage : 0);              // TC: nkb x N x 128 B
   float* sUf = reinterpret_cast<float*>(sU);                        // FMA: N x r floats
   const size_t u_bytes = u_region_bytes<T, TC, N>(a.r);
-  // Owner staging of the chosen buckets' logits: overlays the U operand,
-  // which nothing reads between a step's last MMA and the next gather.
-  T* tbuf = reinterpret_cast<T*>(sU);
-  T* bbuf = tbuf + N * 32;
   // TC: N x N identity (B operand, K-major, 128-byte swizzle) that makes the
   // MMA add each base tile to the bias
   uint8_t* sI = sU + ((u_bytes + 1023) & ~size_t(1023));
   T* sBase = reinterpret_cast<T*>(sI + (TC ? (size_t)N * 128 : 0));  // kNBS x N x 128 tokens
   const size_t base_bytes = (size_t)kNBS * N * kCH * sizeof(T);
   float2* sBucket = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(sBase) + base_bytes);
-  float* zbuf = reinterpret_cast<float*>(sBucket);  // owner staging, after the bucket walk
   Ctl<N>* ctl = reinterpret_cast<Ctl<N>*>(reinterpret_cast<uint8_t*>(sBucket) +
                                           bucket_region_bytes(a.nc, N));
 
@@ -628,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
     const int q4 = warp & 3;         // tensor-memory lane quadrant
     const int n0 = (warp >> 2) * NCOL;  // first column (batch row) of this warp
     uint32_t step_ctr = 0, Lb = 0;
-    uint32_t nbar = 0, tok_expected = 0, rec_expected = 0;
+    uint32_t nbar = 0, rec_expected = 0;
     // Failures are folded into the CTA-wide flag ctl->abort_local; it is only
     // read right after a named barrier, so every compute thread takes the same
     // branch (a waiter that gives up keeps executing until that point).
@@ -857,134 +853,131 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
       cp_async_commit();
     };
 
-    // fin = false: softmax buckets (m, s) in the scale of ctl->M[n];
-    // fin = true: residual / target mass buckets, chosen by ctl->S[n] != 0.
-    auto bucket_mass = [&](int n, int cl, int q, bool fin) {
-      const float2 p = sBucket[((size_t)cl * 4 + q) * N + n];
-      if (!fin) return p.y > 0.f ? p.y * fexp2((p.x - ctl->M[n]) * k) : 0.f;
-      return ctl->S[n] != 0.f ? p.y : p.x;
-    };
-    // Bucket walk for every owned row: warp w walks rows o = w, w + 8, ...
-    // side by side (lanes = buckets, 32 per pass), then loads the logits the
-    // scan of the chosen bucket needs (lanes = its 32 tokens) into tbuf / bbuf:
-    // tgt_row >= 0: that target row (draft steps of a cycle); -1: the stop
-    // row's target and base rows (final step); -2: nothing (drafting only).
-    auto walk_and_assign = [&](bool fin, int g, int tgt_row) {
-      const int n_owned = ctl->n_owned;
-      const int nbk = ncc * 4;  // buckets in ascending token order
-      T tl[kOwnBatch], bl[kOwnBatch];  // logits of the chosen buckets, in flight
-      if (warp < n_owned) {
-        int nn[kOwnBatch], pick[kOwnBatch], lastb[kOwnBatch];
-        float tin[kOwnBatch], carry[kOwnBatch], tin_in[kOwnBatch];
-#pragma unroll
-        for (int j = 0; j < kOwnBatch; ++j) {
-          const int o = warp + 8 * j;
-          const bool has = o < n_owned;
-          nn[j] = ctl->owned[has ? o : warp];
-          tin[j] = has ? ctl->obtarget[o] : 0.f;
-          carry[j] = 0.f;
-          pick[j] = has ? -1 : 0;  // padding slots count as done
-          lastb[j] = -1;
-          tin_in[j] = INFINITY;
-        }
-        for (int b0 = 0; b0 < nbk; b0 += 32) {  // 32 buckets per pass
+    // ---- the draw of one row (stochastic steps and the final step), by the
+    // whole CTA of the row's reducer, from the record ctl->rrec[j]:
+    // 1. warp 0 walks the owner CTA's published bucket statistics in ascending
+    //    token order to the bucket holding the inverse-CDF target;
+    // 2. the bucket's 32 logits are formed here: z = base + U[prev].W with
+    //    the rank split over the 8 warps (the same bf16 inputs as the tensor
+    //    cores, fp32 accumulation);
+    // 3. warp 0 scans the bucket (kind 0: q_i, then the accept test against
+    //    p_i; kind 2: the residual or the bonus row) and writes the outputs.
+    auto draw_row = [&](int kind, int g, int par, int i, int n, int j) {
+      Rec& rr = ctl->rrec[j];
+      if (kind == 0 && (rr.flags & 1)) return;  // the step is redone exactly
+      const int b = g * N + n;
+      const int o = rr.owner;
+      const float M = rr.M;
+      const bool use_p = (rr.flags & 2) != 0;
+      const bool alive = ctl->alive[n] != 0;
+      const int row = kind == 0 ? i : (alive ? K : ctl->stoprow[n]);
+      if (warp == 0) {
+        const int nbk_o = min(a.nc, a.nchunks - o * a.nc) * 4;
+        const float tin = rr.trem;
+        float carry = 0.f, tin_in = INFINITY;
+        int pick = -1, lastb = -1;
+        for (int b0 = 0; b0 < nbk_o && pick < 0; b0 += 32) {  // 32 buckets per pass
           const int bk = b0 + lane;
-          float w[kOwnBatch], incl[kOwnBatch];
-#pragma unroll
-          for (int j = 0; j < kOwnBatch; ++j) {
-            w[j] = bk < nbk ? bucket_mass(nn[j], bk >> 2, bk & 3, fin) : 0.f;
-            incl[j] = w[j];
+          float w = 0.f;
+          if (bk < nbk_o) {
+            const float2 pv = __ldcg(a.gbk + ((size_t)o * a.nbk + bk) * N + n);
+            w = kind == 0 ? (pv.y > 0.f ? pv.y * fexp2((pv.x - M) * k) : 0.f) : (use_p ? pv.y : pv.x);
           }
+          float incl = w;
 #pragma unroll
           for (int off = 1; off < 32; off <<= 1) {
-#pragma unroll
-            for (int j = 0; j < kOwnBatch; ++j) {
-              const float y = __shfl_up_sync(FULL, incl[j], off);
-              if (lane >= off) incl[j] += y;
-            }
+            const float y = __shfl_up_sync(FULL, incl, off);
+            if (lane >= off) incl += y;
           }
-#pragma unroll
-          for (int j = 0; j < kOwnBatch; ++j) {
-            const unsigned cross = __ballot_sync(FULL, carry[j] + incl[j] > tin[j]);
-            const unsigned pos = __ballot_sync(FULL, w[j] > 0.f);
-            const float before = __shfl_sync(FULL, incl[j] - w[j], cross ? __ffs(cross) - 1 : 0);
-            const float total = __shfl_sync(FULL, incl[j], 31);
-            if (pick[j] < 0) {  // uniform across the warp
-              if (pos) lastb[j] = b0 + 31 - __clz(pos);
-              if (cross) {
-                pick[j] = b0 + __ffs(cross) - 1;
-                tin_in[j] = tin[j] - (carry[j] + before);
-              }
-              carry[j] += total;
-            }
+          const unsigned cross = __ballot_sync(FULL, carry + incl > tin);
+          const unsigned pos = __ballot_sync(FULL, w > 0.f);
+          if (pos) lastb = b0 + 31 - __clz(pos);
+          if (cross) {
+            const int l = __ffs(cross) - 1;
+            pick = b0 + l;
+            tin_in = tin - (carry + __shfl_sync(FULL, incl - w, l));
           }
+          carry += __shfl_sync(FULL, incl, 31);
         }
-#pragma unroll
-        for (int j = 0; j < kOwnBatch; ++j) {
-          if (pick[j] < 0) {
-            pick[j] = lastb[j] < 0 ? 0 : lastb[j];
-            tin_in[j] = INFINITY;
-          }
-          const int o = warp + 8 * j;
-          if (lane == 0 && o < n_owned) {
-            ctl->obucket[o] = pick[j];
-            ctl->obtarget[o] = tin_in[j];
-          }
+        if (pick < 0) {
+          pick = lastb < 0 ? 0 : lastb;
+          tin_in = INFINITY;
         }
-#pragma unroll
-        for (int j = 0; j < kOwnBatch; ++j) {  // issued now, used after the staging below
-          const int n = nn[j];
-          const int64_t b = (int64_t)g * N + n;
-          const int v = min((chunk0 + (pick[j] >> 2)) * kCH + (pick[j] & 3) * 32 + lane, V - 1);
-          const int row = tgt_row >= 0 ? tgt_row : (ctl->alive[n] ? K : ctl->stoprow[n]);
-          if (tgt_row != -2) tl[j] = target[(b * (K + 1) + row) * V + v];
-          if (tgt_row == -1) bl[j] = base[(b * K + min(row, K - 1)) * V + v];
+        if (lane == 0) {
+          ctl->dbk = pick;
+          ctl->dtin = tin_in;
         }
       }
       named_sync();
-      // Stage the chosen bucket of every owned row into shared memory, so that
-      // any warp can scan any owned row.  Tensor memory lanes of a quadrant are
-      // reachable only from its two warps, which take alternate rows.
-      {
-        tc_fence_after();
-        const int h = warp >> 2;
-        const bool m0 = lane < n_owned && (ctl->obucket[lane] & 3) == q4;
-        const bool m1 = lane + 32 < n_owned && (ctl->obucket[lane + 32] & 3) == q4;
-        const unsigned q0 = __ballot_sync(FULL, m0), q1 = __ballot_sync(FULL, m1);
-        const unsigned below = (1u << lane) - 1u;
-        const int r0 = __popc(q0 & below), r1 = __popc(q0) + __popc(q1 & below);
-        const unsigned s0 = __ballot_sync(FULL, m0 && (r0 & 1) == h);
-        const unsigned s1 = __ballot_sync(FULL, m1 && (r1 & 1) == h);
-        unsigned long long rem = ((unsigned long long)s1 << 32) | s0;
-        constexpr int SB = 16;  // rows per batch of tensor-memory loads
-        while (rem) {  // warp-uniform
-          int oo[SB];
-          float vv[SB];
-#pragma unroll
-          for (int j = 0; j < SB; ++j) {
-            oo[j] = rem ? __ffsll((long long)rem) - 1 : -1;
-            rem &= rem - 1;
-          }
-#pragma unroll
-          for (int j = 0; j < SB; ++j) {
-            vv[j] = 0.f;
-            if (oo[j] < 0) continue;
-            const int cl = ctl->obucket[oo[j]] >> 2, n = ctl->owned[oo[j]];
-            tmem_ld1(taddr + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(cl * N + n), &vv[j]);
-          }
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < SB; ++j)
-            if (oo[j] >= 0) zbuf[oo[j] * 32 + lane] = vv[j];
+      const int bk = ctl->dbk;
+      const int v0 = (o * a.nc + (bk >> 2)) * kCH + (bk & 3) * 32;
+      const int v = v0 + lane, vc = min(v, V - 1);
+      float tv = 0.f, bv = 0.f;
+      if (warp == 0) {  // the row's logits at the bucket's tokens, in flight meanwhile
+        if (kind == 0) {
+          bv = ld_elem(base, ((int64_t)b * K + i) * V + vc);
+          if (a.mode == MODE_CYCLE) tv = ld_elem(target, ((int64_t)b * (K + 1) + i) * V + vc);
+        } else {
+          tv = ld_elem(target, ((int64_t)b * (K + 1) + row) * V + vc);
+          if (!alive) bv = ld_elem(base, ((int64_t)b * K + row) * V + vc);
         }
       }
-      if (warp < n_owned) {
+      {  // warp w: rank rows [w*ks, w*ks + ks)
+        const int ks = (a.r + 7) / 8, k0 = warp * ks, k1 = min(a.r, k0 + ks);
+        const int prev = ctl->prev[n];
+        const float uval = k0 + lane < k1 ? ld_elem(Ug, (int64_t)prev * a.r + k0 + lane) : 0.f;
+        float wv[32];
 #pragma unroll
-        for (int j = 0; j < kOwnBatch; ++j) {
-          const int o = warp + 8 * j;
-          if (o >= n_owned) continue;
-          if (tgt_row != -2) tbuf[o * 32 + lane] = tl[j];
-          if (tgt_row == -1) bbuf[o * 32 + lane] = bl[j];
+        for (int t = 0; t < 32; ++t) wv[t] = k0 + t < k1 ? ld_elem(Wg, (int64_t)(k0 + t) * V + vc) : 0.f;
+        float part = 0.f;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) part = fmaf(__shfl_sync(FULL, uval, t), wv[t], part);
+        ctl->zpart[warp][lane] = part;
+      }
+      named_sync();
+      if (warp == 0) {
+        float bias = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) bias += ctl->zpart[w][lane];
+        const bool valid = v < V;
+        if (kind == 0) {
+          const float z = bias + bv, S = rr.S;
+          const float e = valid ? fexp2((z - M) * k) : 0.f;
+          const int wl = bucket_scan(e, ctl->dtin);
+          const int d = v0 + wl;
+          const float zd = __shfl_sync(FULL, z, wl), td = __shfl_sync(FULL, tv, wl);
+          const float qd = fexp2((zd - M) * k) / S;
+          const bool test = a.mode == MODE_CYCLE && alive;
+          int accept = 1;
+          float pd = __int_as_float(0x7fc00000);
+          if (test) {
+            pd = fexp2((td - rr.Mt) * k) / rr.St;
+            const float ratio = fexp2(((td - rr.Mt) - (zd - M)) * k) * (S / rr.St);
+            const float uacc =
+                philox_uniform(a.seed, a.cycle, a.row0 + (uint32_t)b, (uint32_t)i, TAG_ACCEPT);
+            accept = uacc < fminf(ratio, 1.0f) ? 1 : 0;
+          }
+          if (lane == 0) {
+            rr.token = d;
+            rr.acc = accept;
+            a.tokens[((int64_t)par * K + i) * N + n] = d;
+            if (a.draft) a.draft[(int64_t)b * K + i] = d;
+            if (a.q_draft) a.q_draft[(int64_t)b * K + i] = qd;
+            if (test) {
+              if (a.p_draft) a.p_draft[(int64_t)b * K + i] = pd;
+              if (accept) a.out[(int64_t)b * (K + 1) + i] = d;
+            }
+          }
+        } else {  // the same expressions as the final epilogue's bucket masses
+          const float4 c = ctl->fcst[n];
+          const float p = fexp2((tv - c.x) * k) * c.y;
+          const float q = c.w != 0.f ? fexp2((bias + bv - c.z) * k) * c.w : 0.f;
+          const float w = valid ? ((alive || use_p) ? p : fmaxf(p - q, 0.f)) : 0.f;
+          const int wl = bucket_scan(w, ctl->dtin);
+          if (lane == 0) {
+            rr.token = v0 + wl;
+            a.out[(int64_t)b * (K + 1) + row] = v0 + wl;
+          }
         }
       }
       named_sync();
@@ -1124,6 +1117,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             }
             rc.tam = ai;
             if (kind == 0) rc.acc = ai == rc.token ? 1 : 0;
+            if (kind == 0 && lane == 0)  // greedy step of a row still verifying
+              a.out[(int64_t)b * (K + 1) + i] = rc.acc ? rc.token : rc.tam;
           } else {
             float Mt = -INFINITY;
 #pragma unroll
@@ -1139,8 +1134,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             rc.St = warp_sum(st);
           }
         }
-        if (lane == 0) store_rec(a.rec + ((int64_t)par * (K + 2) + (kind == 0 ? i : (kind == 1 ? K : K + 1))) * N + n, rc);
+        if (kind == 0 && a.greedy && lane == 0 && a.draft) a.draft[(int64_t)b * K + i] = rc.token;
+        if (lane == 0) ctl->rrec[local] = rc;
       }
+      named_sync();
+      // stochastic draws, one row at a time by the whole CTA
+      if ((kind == 0 && !a.greedy) || kind == 2)
+        for (int j = 0; j < mine; ++j) draw_row(kind, g, par, i, cta + j * G, j);
+      const int slot = kind == 0 ? i : (kind == 1 ? K : K + 1);
+      if (tid < mine)
+        store_rec(a.rec + ((int64_t)par * (K + 2) + slot) * N + (cta + tid * G), ctl->rrec[tid]);
       return mine;
     };
     // publish this CTA's records and wait until every row's record exists
@@ -1199,9 +1202,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
         }
         named_sync();
         gather_u(nb_g);
-        if (!a.greedy && a.mode == MODE_CYCLE && tid < nb_g)  // accept-test uniform of the step
-          ctl->uacc[tid] = philox_uniform(a.seed, a.cycle, a.row0 + (uint32_t)(g * N + tid),
-                                          (uint32_t)i, TAG_ACCEPT);
         // pull the next target row of every live batch row into L2 now; the
         // background pass reads it while this step's barrier completes
         if (a.mode == MODE_CYCLE && tid < nb_g && ctl->alive[tid])
@@ -1283,14 +1283,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               }
               bfly_sum1<NCOL>(d, lane);
               psum += d[0];  // this lane's column, summed over the CTA's chunks
-              if ((lane & (REP - 1)) == 0)
-                bk[n0 + lane / REP] = make_float2(ctl->ref[n0 + lane / REP], d[0]);
+              if ((lane & (REP - 1)) == 0) {
+                const float2 st = make_float2(ctl->ref[n0 + lane / REP], d[0]);
+                bk[n0 + lane / REP] = st;
+                a.gbk[((size_t)cta * a.nbk + cl * 4 + q4) * N + n0 + lane / REP] = st;
+              }
             } else {
               float s[NCOL];
 #pragma unroll
               for (int j = 0; j < NCOL; ++j) s[j] = valid ? 1.f : 0.f;
               bfly_ms<NCOL>(d, s, k, lane);
-              if ((lane & (REP - 1)) == 0) bk[n0 + lane / REP] = make_float2(d[0], s[0]);
+              if ((lane & (REP - 1)) == 0) {
+                bk[n0 + lane / REP] = make_float2(d[0], s[0]);
+                a.gbk[((size_t)cta * a.nbk + cl * 4 + q4) * N + n0 + lane / REP] = make_float2(d[0], s[0]);
+              }
             }
             if (trace && g == 0 && cl < 8 && attempt == 0)
               trace[(size_t)i * kTracePhases + 16 + cl] = globaltimer_ns();
@@ -1355,11 +1361,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             break;
           }
           mark(g, i, 5);
-          // ---------------- row reducers publish one record per row
-          if (tid == 0) {
-            ctl->n_owned = 0;
-            ctl->redo = 0;
-          }
+          // ---------------- row reducers draw the token of their rows and
+          // publish one record per row
+          if (tid == 0) ctl->redo = 0;
           const int mine = reduce_rows(0, g, par, i, nb_g, fast);
           mark(g, i, 12);
           if (!records_hop(mine, nb_g)) {
@@ -1368,29 +1372,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           }
           for (int n = tid; n < nb_g; n += kComputeThreads) {
             const Rec r = load_rec(a.rec + ((int64_t)par * (K + 2) + i) * N + n);
-            const int b = g * N + n;
-            if (a.greedy) {
-              ctl->tok[n] = r.token;
-              if (cta == 0 && a.draft) a.draft[(int64_t)b * K + i] = r.token;
-              if (a.mode == MODE_CYCLE && ctl->alive[n]) {
-                if (cta == 0) a.out[(int64_t)b * (K + 1) + i] = r.acc ? r.token : r.tam;
-                if (!r.acc) {
-                  ctl->alive[n] = 0;
-                  ctl->stoprow[n] = i;
-                }
-              }
-            } else {
+            if (!a.greedy) {
               ctl->M[n] = r.M;
               ctl->S[n] = r.S;
               ctl->ref[n] = r.Mx;
               ctl->Mt[n] = r.Mt;
               ctl->St[n] = r.St;
               if (r.flags & 1) ctl->redo = 1;
-              if (r.owner == cta) {
-                const int slot = atomicAdd(&ctl->n_owned, 1);
-                ctl->owned[slot] = n;
-                ctl->obtarget[slot] = r.trem;
-              }
             }
           }
           named_sync();
@@ -1399,106 +1387,26 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           fast = false;           // exact statistics, re-read from tensor memory
         }
         if (failed) break;
-
-        if (a.greedy) {
-          tc_fence_before();
-          named_sync();
-          if (TC && tid == 0) mbar_arrive(&ctl->tfree);
-        } else {
-          // ---------------- owners: bucket walk, then batched bucket scans
-          walk_and_assign(false, g, a.mode == MODE_CYCLE ? i : -2);
-          mark(g, i, 15);
-          const int n_owned = ctl->n_owned;
-          if (warp < n_owned) {  // owned rows o = warp, warp + 8, ... (n_owned <= N <= 64)
-            int oo[kOwnBatch];
-            float dv[kOwnBatch], td[kOwnBatch], zd[kOwnBatch], qd[kOwnBatch];
-            int dtok[kOwnBatch];
-#pragma unroll
-            for (int j = 0; j < kOwnBatch; ++j) {
-              oo[j] = warp + 8 * j < n_owned ? warp + 8 * j : -1;
-              dtok[j] = 0;
-              dv[j] = oo[j] < 0 ? 0.f : zbuf[oo[j] * 32 + lane];
-            }
-#pragma unroll
-            for (int j = 0; j < kOwnBatch; ++j) {
-              if (oo[j] < 0) continue;
-              const int bk = ctl->obucket[oo[j]], n = ctl->owned[oo[j]];
-              const int v0 = (chunk0 + (bk >> 2)) * kCH + (bk & 3) * 32;  // bucket's first token
-              const float M = ctl->M[n], S = ctl->S[n];
-              const int v = v0 + lane;
-              const bool valid = v < V;
-              const float z = valid ? dv[j] : -INFINITY;  // z = base + bias, kept in tensor memory
-              const float e = valid ? fexp2((z - M) * k) : 0.f;
-              const int wl = bucket_scan(e, ctl->obtarget[oo[j]]);
-              dtok[j] = v0 + wl;
-              zd[j] = __shfl_sync(FULL, z, wl);
-              qd[j] = fexp2((zd[j] - M) * k) / S;
-            }
-            const bool cyc = a.mode == MODE_CYCLE;
-#pragma unroll
-            for (int j = 0; j < kOwnBatch; ++j)  // target logit of the drafted token, staged
-              td[j] = (cyc && oo[j] >= 0) ? to_f<T>(tbuf[oo[j] * 32 + (dtok[j] & 31)]) : 0.f;
-#pragma unroll
-            for (int j = 0; j < kOwnBatch; ++j) {
-              if (oo[j] < 0) continue;
-              const int n = ctl->owned[oo[j]];
-              const int b = g * N + n;
-              const float M = ctl->M[n], S = ctl->S[n];
-              const bool alive = cyc && ctl->alive[n];
-              int accept = 1;
-              float pd = NaNf;
-              if (alive) {
-                const float Mt = ctl->Mt[n], St = ctl->St[n];
-                pd = fexp2((td[j] - Mt) * k) / St;
-                const float ratio = fexp2(((td[j] - Mt) - (zd[j] - M)) * k) * (S / St);
-                accept = ctl->uacc[n] < fminf(ratio, 1.0f) ? 1 : 0;
-              }
-              if (lane == 0) {
-                a.tokens[((int64_t)par * K + i) * N + n] = dtok[j];
-                a.accf[((int64_t)par * K + i) * N + n] = accept;
-                if (a.draft) a.draft[(int64_t)b * K + i] = dtok[j];
-                if (a.q_draft) a.q_draft[(int64_t)b * K + i] = qd[j];
-                if (alive) {
-                  if (a.p_draft) a.p_draft[(int64_t)b * K + i] = pd;
-                  if (accept) a.out[(int64_t)b * (K + 1) + i] = dtok[j];
-                }
-              }
-            }
+        // tensor memory is free for the next step's MMA
+        tc_fence_before();
+        named_sync();
+        if (TC && tid == 0) mbar_arrive(&ctl->tfree);
+        // the step's tokens and accept outcomes, from the records
+        for (int n = tid; n < nb_g; n += kComputeThreads) {
+          const Rec r = load_rec(a.rec + ((int64_t)par * (K + 2) + i) * N + n);
+          ctl->tok[n] = r.token;
+          if (a.mode == MODE_CYCLE && ctl->alive[n] && !r.acc) {
+            ctl->alive[n] = 0;
+            ctl->stoprow[n] = i;
+            ctl->zM[n] = r.M;    // draft statistics of the stop row
+            ctl->zS[n] = r.S;
+            ctl->fMt[n] = r.Mt;  // target statistics of the stop row
+            ctl->fSt[n] = r.St;
           }
-          mark(g, i, 7);
-          tc_fence_before();
-          named_sync();
-          if (TC && tid == 0) mbar_arrive(&ctl->tfree);
-          if (tid == 0) {
-            __threadfence();
-            const int n_owned = ctl->n_owned;
-            if (n_owned) red_release_add_u32(&hdr->tok, (uint32_t)n_owned);
-            tok_expected += (uint32_t)nb_g;
-            if (!grid_wait_count(hdr, &hdr->tok, tok_expected, a.spin, SITE_TOKEN_WAIT) ||
-                ld_volatile_u32(&hdr->abort))
-              ctl->abort_local = 1;
-            __threadfence();
-          }
-          named_sync();
-          mark(g, i, 8);
-          if (ctl->abort_local) {
-            failed = true;
-            break;
-          }
-          for (int n = tid; n < nb_g; n += kComputeThreads) {
-            ctl->tok[n] = __ldcg(a.tokens + ((int64_t)par * K + i) * N + n);
-            if (a.mode == MODE_CYCLE && ctl->alive[n] &&
-                !__ldcg(a.accf + ((int64_t)par * K + i) * N + n)) {
-              ctl->alive[n] = 0;
-              ctl->stoprow[n] = i;
-              ctl->zM[n] = ctl->M[n];  // draft statistics of the stop row
-              ctl->zS[n] = ctl->S[n];
-              ctl->fMt[n] = ctl->Mt[n];  // target statistics of the stop row
-              ctl->fSt[n] = ctl->St[n];
-            }
-          }
-          named_sync();
         }
+        named_sync();
+        mark(g, i, 7);
+        mark(g, i, 8);
         ++step_ctr;
         if (ctl->abort_local) {  // read after the last named barrier of the step
           failed = true;
@@ -1611,7 +1519,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             }
             bfly_sum2<NCOL>(tv, bvv, lane);
             float2* bk = sBucket + ((size_t)cl * 4 + q4) * N;
-            if ((lane & (32 / NCOL - 1)) == 0) bk[n0 + lane / (32 / NCOL)] = make_float2(tv[0], bvv[0]);
+            if ((lane & (32 / NCOL - 1)) == 0) {
+              bk[n0 + lane / (32 / NCOL)] = make_float2(tv[0], bvv[0]);
+              a.gbk[((size_t)cta * a.nbk + cl * 4 + q4) * N + n0 + lane / (32 / NCOL)] =
+                  make_float2(tv[0], bvv[0]);
+            }
             if (trace && g == 0 && cl < 8) trace[(size_t)K * kTracePhases + 16 + cl] = globaltimer_ns();
           }
           if (tid == 0) mbar_arrive(&ctl->ring_free);  // last tile read: slots free
@@ -1642,58 +1554,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             break;
           }
           mark(g, K, 4);
-          if (tid == 0) ctl->n_owned = 0;
+          // the reducers draw each row's residual / bonus token and write it
           const int mine = reduce_rows(2, g, par, K, nb_g, false);
           if (!records_hop(mine, nb_g)) {
             failed = true;
             break;
-          }
-          for (int n = tid; n < nb_g; n += kComputeThreads) {
-            const Rec r = load_rec(a.rec + ((int64_t)par * (K + 2) + K + 1) * N + n);
-            ctl->S[n] = (r.flags & 2) ? 1.f : 0.f;  // which mass the scan uses
-            if (r.owner == cta) {
-              const int slot = atomicAdd(&ctl->n_owned, 1);
-              ctl->owned[slot] = n;
-              ctl->obtarget[slot] = r.trem;
-            }
-          }
-          named_sync();
-          walk_and_assign(true, g, -1);
-          const int n_owned = ctl->n_owned;
-          if (warp < n_owned) {  // owned rows o = warp, warp + 8, ...
-            int oo[kOwnBatch];
-            float dv[kOwnBatch], tvv[kOwnBatch], bvv[kOwnBatch];
-#pragma unroll
-            for (int j = 0; j < kOwnBatch; ++j) {
-              oo[j] = warp + 8 * j < n_owned ? warp + 8 * j : -1;
-              dv[j] = oo[j] < 0 ? 0.f : zbuf[oo[j] * 32 + lane];
-            }
-#pragma unroll
-            for (int j = 0; j < kOwnBatch; ++j) {  // stop rows' logits, staged by the walk
-              const int oj = oo[j] < 0 ? warp : oo[j];  // slot "warp" is owned
-              tvv[j] = to_f<T>(tbuf[oj * 32 + lane]);
-              bvv[j] = to_f<T>(bbuf[oj * 32 + lane]);
-            }
-#pragma unroll
-            for (int j = 0; j < kOwnBatch; ++j) {
-              if (oo[j] < 0) continue;
-              const int bk = ctl->obucket[oo[j]], n = ctl->owned[oo[j]];
-              const int v0 = (chunk0 + (bk >> 2)) * kCH + (bk & 3) * 32;
-              const int b = g * N + n;
-              const bool use_p = ctl->S[n] != 0.f;
-              const bool bonus = ctl->alive[n] != 0;
-              const int row = bonus ? K : ctl->stoprow[n];
-              const int v = v0 + lane;
-              float w = 0.f;
-              if (v < V) {  // the same expressions as the final epilogue's bucket masses
-                const float4 c = ctl->fcst[n];
-                const float p = fexp2((tvv[j] - c.x) * k) * c.y;
-                const float q = c.w != 0.f ? fexp2((dv[j] + bvv[j] - c.z) * k) * c.w : 0.f;
-                w = (bonus || use_p) ? p : fmaxf(p - q, 0.f);
-              }
-              const int wl = bucket_scan(w, ctl->obtarget[oo[j]]);
-              if (lane == 0) a.out[(int64_t)b * (K + 1) + row] = v0 + wl;
-            }
           }
           mark(g, K, 5);
           tc_fence_before();
@@ -1823,17 +1688,19 @@ namespace {
 size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 }  // namespace
 
-// Workspace body: trace | dpart | tpart | tokens | accf | records, each 256-byte aligned.
+// Workspace body: trace | dpart | tpart | tokens | records | bucket statistics,
+// each 256-byte aligned.
 size_t cycle_trace_bytes(int K) { return a256(sizeof(uint64_t) * (size_t)(K + 2) * kTracePhases); }
 namespace {
 size_t dpart_bytes(int K, int N) { return a256(sizeof(float4) * 2 * (size_t)(K + 1) * N * kMaxG); }
 size_t tpart_bytes(int K, int N) { return a256(sizeof(float2) * 2 * (size_t)(K + 1) * N * kMaxG); }
 size_t tok_bytes(int K, int N) { return a256(sizeof(int32_t) * 2 * (size_t)K * N); }
 size_t rec_bytes(int K, int N) { return a256(sizeof(Rec) * 2 * (size_t)(K + 2) * N); }
+size_t gbk_bytes(const CycleGeom& g) { return a256(sizeof(float2) * (size_t)g.G * g.nc * 4 * g.N); }
 }  // namespace
 size_t cycle_ws_bytes(int K, const CycleGeom& g) {
-  return cycle_trace_bytes(K) + dpart_bytes(K, g.N) + tpart_bytes(K, g.N) + 2 * tok_bytes(K, g.N) +
-         rec_bytes(K, g.N);
+  return cycle_trace_bytes(K) + dpart_bytes(K, g.N) + tpart_bytes(K, g.N) + tok_bytes(K, g.N) +
+         rec_bytes(K, g.N) + gbk_bytes(g);
 }
 
 cudaError_t launch_cycle(const CycleLaunch& L, const CycleGeom& g, WsHeader* hdr, uint8_t* body,
@@ -1862,9 +1729,10 @@ cudaError_t launch_cycle(const CycleLaunch& L, const CycleGeom& g, WsHeader* hdr
   body += tpart_bytes(L.K, g.N);
   a.tokens = reinterpret_cast<int32_t*>(body);
   body += tok_bytes(L.K, g.N);
-  a.accf = reinterpret_cast<int32_t*>(body);
-  body += tok_bytes(L.K, g.N);
   a.rec = reinterpret_cast<Rec*>(body);
+  body += rec_bytes(L.K, g.N);
+  a.gbk = reinterpret_cast<float2*>(body);
+  a.nbk = g.nc * 4;
   a.B = L.B;
   a.K = L.K;
   a.V = L.V;

@@ -342,12 +342,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, bo
 // Arrive (release) and wait (acquire) until `target` arrivals; one thread per CTA.
 SPEC_DEV bool grid_wait_count(WsHeader* h, const uint32_t* counter, uint32_t target,
                               uint64_t limit, int32_t site) {
-  uint32_t backoff = 32;
   for (uint64_t it = 0; it < limit; ++it) {
-    if (ld_acquire_u32(counter) >= target) return true;
-    if (ld_volatile_u32(&h->abort)) return false;
-    __nanosleep(backoff);
-    if (backoff < 256) backoff <<= 1;
+    // both loads in flight together: the abort flag first (relaxed), then the
+    // counter (acquire, which orders only what follows it)
+    const uint32_t ab = ld_volatile_u32(&h->abort);
+    const uint32_t c = ld_acquire_u32(counter);
+    if (ab) return false;
+    if (c >= target) return true;
+    __nanosleep(32);
   }
   record_error(h, SPEC_ERR_TIMEOUT, site, (int32_t)target, (int32_t)ld_volatile_u32(counter));
   return false;

@@ -636,13 +636,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
     auto grid_barrier = [&]() {  // all compute threads call it
       named_sync();
       if (tid == 0) {
-        __threadfence();
+        // the barrier above orders the CTA's writes before this release
         red_release_add_u32(&hdr->bar, 1u);
         ++nbar;
-        if (!grid_wait_count(hdr, &hdr->bar, nbar * (uint32_t)G, a.spin, SITE_GRID_BARRIER) ||
-            ld_volatile_u32(&hdr->abort))
+        if (!grid_wait_count(hdr, &hdr->bar, nbar * (uint32_t)G, a.spin, SITE_GRID_BARRIER))
           ctl->abort_local = 1;
-        __threadfence();
       }
       named_sync();
       return ctl->abort_local == 0;
@@ -651,17 +649,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
     auto grid_arrive = [&]() {
       named_sync();
       if (tid == 0) {
-        __threadfence();
+        // the barrier above orders the CTA's writes before this release
         red_release_add_u32(&hdr->bar, 1u);
         ++nbar;
       }
     };
     auto grid_wait = [&]() {
       if (tid == 0) {
-        if (!grid_wait_count(hdr, &hdr->bar, nbar * (uint32_t)G, a.spin, SITE_GRID_BARRIER) ||
-            ld_volatile_u32(&hdr->abort))
+        if (!grid_wait_count(hdr, &hdr->bar, nbar * (uint32_t)G, a.spin, SITE_GRID_BARRIER))
           ctl->abort_local = 1;
-        __threadfence();
       }
       named_sync();
       return ctl->abort_local == 0;
@@ -865,6 +861,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
     auto draw_row = [&](int kind, int g, int par, int i, int n, int j) {
       Rec& rr = ctl->rrec[j];
       if (kind == 0 && (rr.flags & 1)) return;  // the step is redone exactly
+      const bool tr = kind == 0 && j == 0;
       const int b = g * N + n;
       const int o = rr.owner;
       const float M = rr.M;
@@ -909,6 +906,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
         }
       }
       named_sync();
+      if (tr) mark(g, i, 14);
       const int bk = ctl->dbk;
       const int v0 = (o * a.nc + (bk >> 2)) * kCH + (bk & 3) * 32;
       const int v = v0 + lane, vc = min(v, V - 1);
@@ -935,6 +933,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
         ctl->zpart[warp][lane] = part;
       }
       named_sync();
+      if (tr) mark(g, i, 15);
       if (warp == 0) {
         float bias = 0.f;
 #pragma unroll
@@ -1138,6 +1137,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
         if (lane == 0) ctl->rrec[local] = rc;
       }
       named_sync();
+      if (kind == 0) mark(g, i, 13);
       // stochastic draws, one row at a time by the whole CTA
       if ((kind == 0 && !a.greedy) || kind == 2)
         for (int j = 0; j < mine; ++j) draw_row(kind, g, par, i, cta + j * G, j);
@@ -1150,13 +1150,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
     auto records_hop = [&](int mine, int nb_g) {
       named_sync();
       if (tid == 0) {
-        __threadfence();
         if (mine) red_release_add_u32(&hdr->rec, (uint32_t)mine);
         rec_expected += (uint32_t)nb_g;
-        if (!grid_wait_count(hdr, &hdr->rec, rec_expected, a.spin, SITE_REC_WAIT) ||
-            ld_volatile_u32(&hdr->abort))
+        if (!grid_wait_count(hdr, &hdr->rec, rec_expected, a.spin, SITE_REC_WAIT))
           ctl->abort_local = 1;
-        __threadfence();
       }
       named_sync();
       return ctl->abort_local == 0;
@@ -1214,7 +1211,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
         bool fast = !a.greedy && i > 0;
         for (int attempt = 0; attempt < 2; ++attempt) {
           // ---------------- epilogue: z = base + bias, bucket statistics
-          uint64_t t_wait = 0, t_base = 0, t_st = 0;
+          uint64_t t_wait = 0;
           float psum = 0.f;
           float rmax[NCOL];
 #pragma unroll
@@ -1231,10 +1228,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
               if (trace) t_wait += globaltimer_ns() - t_w0;
               if (!TC) {
                 const uint32_t bslot = Lb % kNBS;
-                const uint64_t t_b0 = trace ? globaltimer_ns() : 0;
                 if (!mbar_wait_bounded(&ctl->bfull[bslot], (Lb / kNBS) & 1, a.spin, &hdr->abort))
                   soft_fail(SPEC_ERR_TIMEOUT, SITE_MBAR_BASE, cta, i);
-                if (trace) t_base += globaltimer_ns() - t_b0;
                 const T* bt = sBase + (size_t)bslot * N * kCH;
 #pragma unroll
                 for (int j = 0; j < NCOL; ++j) d[j] += to_f<T>(bt[(n0 + j) * kCH + vl]);
@@ -1252,9 +1247,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
                 }
               }
               // z replaces the bias in tensor memory: owner scans (and a redo) read it
-              const uint64_t t_s0 = trace ? globaltimer_ns() : 0;
               if (!TC && !a.greedy) tmem_st_cols<NCOL>(tcol, d);  // TC: z is in tensor memory
-              if (trace) t_st += globaltimer_ns() - t_s0;
             } else {
               tmem_ld_cols<NCOL>(tcol, d);  // z of this step, kept in tensor memory
 #pragma unroll
@@ -1312,10 +1305,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           named_sync();
           tc_fence_after();
           mark(g, i, 2);
+          if (a.trace && g == 0 && tid == 0 && attempt == 0)
+            atomicMax(reinterpret_cast<unsigned long long*>(a.trace) + (size_t)i * kTracePhases + 8,
+                      (unsigned long long)globaltimer_ns());
           if (trace && g == 0) {
             trace[(size_t)i * kTracePhases + 11] = t_wait;
-            trace[(size_t)i * kTracePhases + 13] = t_base;
-            trace[(size_t)i * kTracePhases + 14] = t_st;
           }
           // ---------------- CTA partial per batch row
           if (fast) {  // common reference: the four quadrants' running sums
@@ -1366,6 +1360,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           if (tid == 0) ctl->redo = 0;
           const int mine = reduce_rows(0, g, par, i, nb_g, fast);
           mark(g, i, 12);
+          // timeline: the last reducer and the last epilogue over all CTAs
+          if (a.trace && g == 0 && tid == 0) {
+            if (mine) atomicMax(reinterpret_cast<unsigned long long*>(a.trace) + (size_t)i * kTracePhases + 7,
+                                (unsigned long long)globaltimer_ns());
+          }
           if (!records_hop(mine, nb_g)) {
             failed = true;
             break;
@@ -1405,8 +1404,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           }
         }
         named_sync();
-        mark(g, i, 7);
-        mark(g, i, 8);
         ++step_ctr;
         if (ctl->abort_local) {  // read after the last named barrier of the step
           failed = true;

@@ -1180,7 +1180,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
       }
       named_sync();
       mark(g, K + 1, 0);
-      if (a.mode == MODE_CYCLE) target_row_stats(g, par, 0, nb_g);
       mark(g, K + 1, 1);
 
       for (int i = 0; i < K; ++i) {
@@ -1199,12 +1198,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
         }
         named_sync();
         gather_u(nb_g);
-        // pull the next target row of every live batch row into L2 now; the
-        // background pass reads it while this step's barrier completes
+        // pull the next target row of every live batch row into L2 for the next
+        // step, and take this step's target row statistics while the tensor
+        // cores run the bias (the epilogue would only wait for them)
         if (a.mode == MODE_CYCLE && tid < nb_g && ctl->alive[tid])
           prefetch_l2_bulk(target + ((int64_t)(g * N + tid) * (K + 1) + i + 1) * V + vslice_lo,
                            (uint32_t)((vslice_hi - vslice_lo) * sizeof(T)));
         mark(g, i, 1);
+        if (a.mode == MODE_CYCLE) target_row_stats(g, par, i, nb_g);
 
         // From step 1 on the softmax partials share a per-row reference (the
         // previous step's true max), so bucket statistics are plain sums.
@@ -1347,8 +1348,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           }
           grid_arrive();
           mark(g, i, 3);
-          // background while the barrier completes: next target row, rows alive so far
-          if (attempt == 0 && a.mode == MODE_CYCLE) target_row_stats(g, par, i + 1, nb_g);
           mark(g, i, 4);
           if (!grid_wait()) {
             failed = true;
@@ -1429,8 +1428,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
       }
 
       if (a.mode == MODE_CYCLE) {
-        // row-K target partials (written after the last barrier) become visible
+        if (!a.greedy) {
+          // ---------------- final step: residual at the stop row, or the bonus.
+          // U rows at each row's stop position first, so the bias MMA runs
+          // while row K's target statistics and their exchange complete.
+          for (int n = tid; n < N; n += kComputeThreads) {
+            int p = 0;
+            if (n < nb_g && !ctl->alive[n]) {
+              const int j = ctl->stoprow[n];
+              p = j == 0 ? __ldg(a.last_token + g * N + n)
+                         : __ldcg(a.tokens + ((int64_t)par * K + (j - 1)) * N + n);
+              if (p < 0 || p >= V) p = 0;
+            }
+            ctl->prev[n] = p;
+          }
+          named_sync();
+          gather_u(nb_g);
+        }
         mark(g, K, 0);
+        target_row_stats(g, par, K, nb_g);  // row K of the rows that accepted every draft
         if (!grid_barrier()) {
           failed = true;
           break;
@@ -1455,22 +1471,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
           named_sync();
         }
         if (!a.greedy) {
-          // ---------------- final step: residual at the stop row, or the bonus
-          for (int n = tid; n < N; n += kComputeThreads) {
-            int p = 0;
-            if (n < nb_g && !ctl->alive[n]) {
-              const int j = ctl->stoprow[n];
-              p = j == 0 ? __ldg(a.last_token + g * N + n)
-                         : __ldcg(a.tokens + ((int64_t)par * K + (j - 1)) * N + n);
-              if (p < 0 || p >= V) p = 0;
-            }
-            ctl->prev[n] = p;
-            if (n < nb_g)  // final-row constants, read once per column and chunk
-              ctl->fcst[n] = make_float4(ctl->fMt[n], 1.f / ctl->fSt[n], ctl->zM[n],
-                                         ctl->alive[n] ? 0.f : 1.f / ctl->zS[n]);
-          }
+          for (int n = tid; n < nb_g; n += kComputeThreads)  // final-row constants
+            ctl->fcst[n] = make_float4(ctl->fMt[n], 1.f / ctl->fSt[n], ctl->zM[n],
+                                       ctl->alive[n] ? 0.f : 1.f / ctl->zS[n]);
           named_sync();
-          gather_u(nb_g);
           mark(g, K, 2);
           uint64_t t_fmma = 0, t_ftile = 0;
           for (int cl = 0; cl < ncc; ++cl) {

@@ -1088,6 +1088,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             const float bown = __shfl_sync(FULL, before, fb ? 0 : own / E);
             rc.owner = fb ? max(lp, 0) : own;
             rc.trem = fb ? INFINITY : tgt - bown;
+
             rc.M = M;
             rc.S = total;
             rc.Mx = mx;

@@ -282,6 +282,31 @@ def test_cycle_target_equals_draft_accepts_everything():
         assert np.array_equal(g["out"][:, : w.K], g["draft"])
 
 
+def test_cycle_reference_jump_takes_the_exact_round():
+    """From step 1 on the bucket sums are taken relative to the previous
+    step's max.  A +120 spike in row 1 of half the batch rows makes that
+    reference far too low at step 1 (and far too high at step 2, where the
+    sums underflow): the reducers must ask for the exact round, and the draws
+    must still be the oracle's."""
+    w = synth.Workload("jump", B=20, K=5, V=3000, r=64, dtype="bf16", sigma=0.6, seed=66,
+                       uw_std=0.3)
+    d = synth.make(w)
+    base = d["base"].float()
+    for b in range(0, w.B, 2):
+        base[b, 1, (37 * b + 11) % w.V] += 120.0
+    d["base"] = base.to(torch.bfloat16).contiguous()
+    total_flag = 0
+    for cyc in range(3):
+        g = gpu_cycle(w, d, T=1.0, seed=23, cyc=cyc)
+        o = orc_cycle(w, d, T=1.0, seed=23, cyc=cyc)
+        total_flag += compare_cycle(g, o, w.K)
+        check_invariants(g["out"], g["tau"], g["draft"], w.K)
+        # the spiked rows draft their spike at step 1 (probability ~1)
+        for b in range(0, w.B, 2):
+            assert g["draft"][b, 1] == (37 * b + 11) % w.V
+    assert total_flag <= max(1, 3 * w.B // 10)
+
+
 @pytest.mark.parametrize("cfg,rows", [("c3", [0, 1, 2, 63]), ("c4", [0, 255]), ("c5", [0, 127])])
 def test_cycle_full_size_sampled_rows(cfg, rows):
     """Full-size launch (the benchmark's configuration); the oracle checks

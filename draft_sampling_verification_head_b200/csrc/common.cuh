@@ -24,7 +24,7 @@ struct WsHeader {
   int32_t err_a;        // diagnostic values
   int32_t err_b;
   uint32_t bar;         // grid-barrier arrivals in the current launch
-  uint32_t tok;         // tokens published in the current launch
+  uint32_t spare;       // unused
   uint32_t exit_count;  // CTAs that finished the current launch
   uint32_t abort;       // nonzero once a CTA of the current launch gave up
   uint32_t rec;         // row records published in the current launch
@@ -35,7 +35,7 @@ static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 enum ErrSite : int32_t {
   SITE_NONE = 0,
   SITE_GRID_BARRIER = 1,
-  SITE_TOKEN_WAIT = 2,
+  SITE_UNUSED_2 = 2,
   SITE_MBAR_FULL = 3,
   SITE_MBAR_MMA = 4,
   SITE_MBAR_BASE = 5,

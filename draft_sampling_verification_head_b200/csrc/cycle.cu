@@ -149,19 +149,16 @@ SPEC_DEV Rec load_rec(const Rec* src) {
   return r;
 }
 
-// Shared region of the MMA's U operand (tensor cores: bf16 rows in k-blocks;
-// otherwise fp32 rows), reused for the owners' staged logits.
+// Shared region of the MMA's U operand: tensor cores, bf16 rows in 64-wide
+// k-blocks; otherwise fp32 rows.
 template <typename T, bool TC, int N>
 __host__ __device__ inline size_t u_region_bytes(int r) {
-  const size_t u = TC ? (size_t)(r / 64) * N * 128 : (size_t)N * r * 4;
-  const size_t st = (size_t)2 * N * 32 * sizeof(T);
-  return u > st ? u : st;
+  return TC ? (size_t)(r / 64) * N * 128 : (size_t)N * r * 4;
 }
 
-// Shared region for per-bucket statistics, reused to stage owned rows' values.
+// Shared region for the CTA's per-bucket statistics of one step.
 __host__ __device__ inline size_t bucket_region_bytes(int nc, int N) {
-  const size_t b = (size_t)nc * 4 * N * sizeof(float2), z = (size_t)N * 32 * sizeof(float);
-  return b > z ? b : z;
+  return (size_t)nc * 4 * N * sizeof(float2);
 }
 
 SPEC_DEV void named_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
@@ -1601,7 +1598,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
     if (prior == (uint32_t)G - 1) {
       __threadfence();
       hdr->bar = 0;
-      hdr->tok = 0;
       hdr->rec = 0;
       hdr->abort = 0;
       __threadfence();

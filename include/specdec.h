@@ -19,7 +19,7 @@
  *   p = softmax(target / T), q = softmax((base + bias) / T).
  *
  * Random numbers: Philox4x32-10 (Salmon et al., SC'11), key = seed,
- * counter = (position, batch row, lo32(cycle), tag | bits 32..47 of cycle << 16),
+ * counter = (position, row_offset + batch row, lo32(cycle), tag | bits 32..47 of cycle << 16),
  * word 0 mapped to [0,1) as (x >> 8) * 2^-24; tag 0 = draft draw, 1 = accept
  * test, 2 = residual or bonus draw.  Sampling is by inverse CDF in ascending
  * token order: the first token whose inclusive prefix mass exceeds u * total.
@@ -89,7 +89,7 @@ typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 
 typedef struct {
   int32_t B;             /* batch rows, >= 1 */
-  int32_t K;             /* draft block length, 1 .. 64 */
+  int32_t K;             /* draft block length, 1 .. 1024 */
   int32_t V;             /* vocabulary, >= 1; bf16 needs V % 8 == 0, f32 V % 4 == 0 */
   int32_t r;             /* Markov rank: 0 (no head) or 1..256; bf16 tensor-core path needs r % 64 == 0 */
   int32_t dtype;         /* spec_dtype of base, target, U, W */

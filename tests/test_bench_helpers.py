@@ -1,0 +1,65 @@
+"""Host-side pieces of bench.py (CPU only): the roofline byte counts, the clock
+sampler's windowing and the peak / traffic lookups."""
+import json
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import synth  # noqa: E402
+
+
+def test_full_stream_bytes_config3():
+    # K draft rows + K+1 target rows of bf16 logits, W once, the gathered U rows
+    w = synth.WORKLOADS["c3"]
+    assert bench.full_stream_bytes(w) == 2 * 64 * 33 * 129280 + 2 * 256 * 129280 + 2 * 64 * 16 * 256
+    assert bench.full_stream_bytes(w) == 612794368
+
+
+def test_early_exit_bytes_bounds():
+    w = synth.WORKLOADS["c3"]
+    full = bench.full_stream_bytes(w)
+    assert bench.early_exit_bytes(w, np.full(w.B, w.K + 1)) == full
+    one = bench.early_exit_bytes(w, np.ones(w.B, dtype=np.int64))
+    assert one == 2 * (w.B * w.K + w.B) * w.V + 2 * w.r * w.V + 2 * w.B * w.K * w.r
+    assert one < full
+
+
+def test_clock_sampler_keeps_the_timed_window_only():
+    c = bench.ClockSampler(0)
+    row = lambda mhz, reason: ["0", str(mhz), "1965", "300.0", "0x0", "Not Active", "Not Active",
+                               "Not Active", reason]
+    c.samples = [(1.0, row(900, "Not Active")), (2.0, row(1965, "Not Active")),
+                 (3.0, row(1950, "Active")), (9.0, row(600, "Not Active"))]
+    c.t0, c.t1 = 1.5, 3.5
+    s = c.summary()
+    assert s["samples"] == 2
+    assert s["sm_mhz"] == (1965 + 1950) / 2
+    assert s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_sampler_without_samples_says_so():
+    c = bench.ClockSampler(0)
+    c.t0, c.t1 = 0.0, 1.0
+    assert c.summary()["reasons"] == ["unsampled"]
+
+
+def test_measured_peak_reads_the_driver_file():
+    peak, kind = bench.measured_peak()
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        assert kind == "measured" and peak == float(json.load(open(p))["hbm_gbs"])
+    else:
+        assert kind == "fallback" and peak == 6650.0
+
+
+def test_recorded_traffic_only_for_the_profiled_source():
+    assert bench.recorded_traffic("not-the-profiled-source") is None
+    p = os.path.join(ROOT, "profiles", "k_cycle_c3_ncu.json")
+    d = json.load(open(p))
+    assert bench.recorded_traffic(d["csrc_hash"]) == d["dram_bytes_per_launch"]

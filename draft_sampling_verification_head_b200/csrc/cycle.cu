@@ -11,26 +11,29 @@
 // Design (one launch, one CTA per SM, cooperative so all CTAs are resident):
 //  * The vocabulary is cut into 128-token chunks; CTA c owns nc consecutive
 //    chunks for the whole launch.  Batch rows are processed in groups of N
-//    (16/32/64) = the tcgen05 N dimension.
-//  * Per draft step, per chunk: the bias tile D[v, b] = W^T[v, :] . U[prev_b]^T
-//    is one tcgen05.mma chain (M = 128 tokens, N batch rows, K = r) into tensor
-//    memory; W^T streams through an 8-stage TMA ring (128-byte swizzle, L2
-//    evict-last), the gathered U rows form the swizzled K-major B operand, and
-//    the base logit tile arrives by TMA.  D stays in tensor memory for the whole
-//    step (nc * N <= 512 columns), so the owner of a sample can re-read it.
-//  * The epilogue adds the base tile and reduces softmax statistics of
-//    z / T per 32-token bucket with a transposing butterfly (one exp2 per
-//    element), then per CTA; the (m, s) partials are exchanged through global
-//    memory behind a grid barrier.  Every CTA combines all partials in the same
-//    fixed order, so all agree on Z, on the prefix masses and on which CTA owns
-//    the inverse-CDF draw; the owner walks its buckets and scans one bucket with
-//    a warp prefix sum.  Greedy steps take the arg-max instead (no owner step).
-//  * Cycle mode verifies on the fly: while waiting at each grid barrier the
-//    CTAs stream the next target row for the rows still alive (early exit: a
-//    row is never read past its first rejection), and the owner of d_i decides
-//    the accept test with p_i(d_i) / q_i(d_i).  A last step recomputes the bias
-//    of each row's stop position and draws the residual max(p - q, 0) (or the
-//    bonus from target row K) with the same two-level inverse CDF.
+//    (16/32/64) = the tcgen05 N dimension.  Warps: 8 compute warps, a W TMA
+//    producer, the MMA issuer and a base-tile producer.
+//  * Per draft step, per chunk: D[v, b] = W^T[v, :] . U[prev_b]^T + base[b, v]
+//    is one tcgen05.mma chain into tensor memory (M = 128 tokens, N batch rows,
+//    K = r, then N more K-rows that add the base tile against an identity):
+//    W^T streams through a TMA ring (128-byte swizzle, L2 evict-last), the
+//    gathered U rows form the swizzled K-major B operand, the base tile
+//    arrives by TMA.  Meanwhile the compute warps take the target row's
+//    statistics over the CTA's slice.
+//  * The epilogue reduces softmax statistics of z / T per 32-token bucket with
+//    a transposing butterfly (one exp2 per element; from step 1 on as plain
+//    sums against the previous step's max), publishes them per bucket and per
+//    CTA, and meets the other CTAs at a grid barrier.
+//  * Row n's reducer (CTA n mod G) combines the per-CTA partials in ascending
+//    token order, finds the CTA and then the bucket holding the inverse-CDF
+//    target, forms that bucket's 32 logits from the bf16 inputs with the whole
+//    CTA, scans them, runs the accept test with p_i(d_i) / q_i(d_i) and writes
+//    the outputs and a 48-byte record; a counter hands the records to every
+//    CTA.  Greedy steps take the arg-max instead.
+//  * Verification runs on the fly (early exit: a row's target rows are never
+//    read past its first rejection).  A last step recomputes the bias at each
+//    row's stop position, gathers the stop rows' logits and draws the residual
+//    max(p - q, 0) (or the bonus from target row K) the same way.
 //  * Every wait is bounded (spin limit); a CTA that gives up records
 //    SPEC_ERR_TIMEOUT in the workspace, the others notice and all exit.
 #include <algorithm>
@@ -805,7 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
       }
     };
 
-    // Owner scan of one 32-token bucket (whole warp): weights per lane, target
+    // Scan of one 32-token bucket (whole warp): weights per lane, target
     // tin within the bucket; returns the winning lane.
     auto bucket_scan = [&](float wv, float tin) {
       float incl = wv;
@@ -981,8 +984,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
 
     // ---- row reducers.  Row n of a group is combined by one warp of CTA
     // n % G; lanes hold E consecutive per-CTA partials each, so a warp prefix
-    // sum walks the CTAs in ascending token order.  The reducer alone decides
-    // the owner CTA of the row's inverse-CDF draw and publishes a record.
+    // sum walks the CTAs in ascending token order.  The reducer finds the CTA
+    // holding the row's inverse-CDF target, draws the token (draw_row) and
+    // publishes a record.
     //  kind 0: draft step i -- stochastic: scale, total, owner, residual target,
     //          true max; greedy: the arg-max token; plus target row i
     //          statistics (or arg-max and the accept outcome) for live rows;
@@ -1245,7 +1249,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
                   if (n0 + j < nb_g) a.biased_out[((int64_t)b * K + i) * V + v] = d[j];
                 }
               }
-              // z replaces the bias in tensor memory: owner scans (and a redo) read it
+              // fp32 path: z replaces the bias in tensor memory for a redo
               if (!TC && !a.greedy) tmem_st_cols<NCOL>(tcol, d);  // TC: z is in tensor memory
             } else {
               tmem_ld_cols<NCOL>(tcol, d);  // z of this step, kept in tensor memory

@@ -33,10 +33,22 @@ METRIC = "draft+verify positions/sec and HBM GB/s vs B200 peak at B=64 K=16 V=12
 WORKLOAD = "c3"
 
 
-def csrc_hash() -> str:
+def _strip_comments(src: str) -> str:
+    """C/C++ source without comments or blank lines (string literals in the
+    kernels hold no comment markers)."""
+    import re
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(l.rstrip() for l in src.splitlines() if l.strip())
+
+
+def csrc_hash(root: str = ROOT) -> str:
+    """Fingerprint of the kernel sources, comments excluded: a recorded ncu
+    traffic figure stays valid while the code it measured is unchanged."""
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "draft_sampling_verification_head_b200", "csrc", "*"))):
-        h.update(open(f, "rb").read())
+    for f in sorted(glob.glob(os.path.join(root, "draft_sampling_verification_head_b200", "csrc", "*"))):
+        h.update(os.path.basename(f).encode())
+        h.update(_strip_comments(open(f, encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 

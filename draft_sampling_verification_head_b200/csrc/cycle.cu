@@ -743,9 +743,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
             ms_combine(m[r], s[r], m2, s2, k);
             amax_combine(av[r], ai[r], a2, i2);
           }
-          if (lane == 0)
+          if (lane == 0) {
             a.tpart[(((int64_t)par * (K + 1) + row) * N + rn[r]) * kMaxG + cta] =
                 a.greedy ? make_float2(av[r], __int_as_float(ai[r])) : make_float2(m[r], s[r]);
+            // step 0: the CTA's target max is its reference for the draft sums
+            if (row == 0 && !a.greedy) ctl->ref[rn[r]] = m[r];
+          }
         }
       }
     };
@@ -1208,10 +1211,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle(const __grid_constant__ A
                            (uint32_t)((vslice_hi - vslice_lo) * sizeof(T)));
         mark(g, i, 1);
         if (a.mode == MODE_CYCLE) target_row_stats(g, par, i, nb_g);
+        if (i == 0) named_sync();  // step 0's references, written above
 
-        // From step 1 on the softmax partials share a per-row reference (the
-        // previous step's true max), so bucket statistics are plain sums.
-        bool fast = !a.greedy && i > 0;
+        // The bucket statistics are plain sums against a per-row reference:
+        // the previous step's true max (all CTAs alike), or at step 0 of a
+        // cycle this CTA's max of target row 0 (partials carry their own
+        // reference, so CTAs may differ).  Drafting alone starts exactly.
+        bool fast = !a.greedy && (i > 0 || a.mode == MODE_CYCLE);
         for (int attempt = 0; attempt < 2; ++attempt) {
           // ---------------- epilogue: z = base + bias, bucket statistics
           uint64_t t_wait = 0;

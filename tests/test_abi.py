@@ -49,6 +49,8 @@ def _p(**kw):
     (dict(temperature=0.0), sd.SPEC_ERR_INVALID_ARG),
     (dict(V=1001), sd.SPEC_ERR_UNSUPPORTED),
     (dict(row_offset=2**31 - 3), sd.SPEC_ERR_INVALID_ARG),  # row_offset + B beyond 2^31
+    (dict(K=1025), sd.SPEC_ERR_INVALID_ARG),
+    (dict(r=-1), sd.SPEC_ERR_INVALID_ARG),
 ])
 def test_host_validation_before_launch(kw, code):
     L = sd.lib()
@@ -113,3 +115,19 @@ def test_params_offsets_match_the_c_compiler(tmp_path):
                                           text=True).stdout.split()]
     want = [ctypes.sizeof(sd.SpecParams)] + [getattr(sd.SpecParams, n).offset for n in names]
     assert got == want
+
+
+def test_valid_params_pass_host_validation():
+    """Greedy needs no temperature, and the largest row offset that still fits
+    is accepted: validation passes and the call only fails for want of a GPU
+    (or launches, on a machine that has one)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present: the call would launch")
+    L = sd.lib()
+    fake = ctypes.c_void_p(0x1000)
+    for kw in (dict(greedy=True, temperature=0.0), dict(row_offset=2**31 - 4)):
+        p = _p(**kw).c()
+        rc = L.spec_cycle(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, None,
+                          None, fake, None)
+        assert rc not in (sd.SPEC_ERR_INVALID_ARG, sd.SPEC_ERR_UNSUPPORTED), (kw, rc)

@@ -57,6 +57,60 @@ def test_philox_uniformity_chi2(orc):
     assert np.all(np.abs(bits - 0.5) < 5 * 0.5 / math.sqrt(len(words)))
 
 
+def _curand_host_lib():
+    """The CUDA toolkit's cuRAND library (its host generators need no GPU)."""
+    import ctypes
+    import glob
+    cands = ["/usr/local/cuda/lib64/libcurand.so", "/usr/local/cuda/lib64/libcurand.so.10"]
+    try:
+        import nvidia.curand  # pip wheel shipped with torch
+        cands += glob.glob(os.path.join(list(nvidia.curand.__path__)[0], "lib", "libcurand.so*"))
+    except ImportError:
+        pass
+    for c in cands:
+        if os.path.exists(c):
+            try:
+                return ctypes.CDLL(c)
+            except OSError:
+                pass
+    return None
+
+
+def test_philox_matches_curand_host_generator(orc):
+    """Philox4x32-10 (Salmon et al., SC'11) as written in the oracle against an
+    independent implementation of the same published generator: cuRAND's host
+    generator CURAND_RNG_PSEUDO_PHILOX4_32_10, which runs on the CPU.  Its
+    stream emits block j (four 32-bit words) from counter (0, 0, j, 0) under
+    key (lo32(seed), hi32(seed)), and a generator offset of 4j starts at block
+    j, for the first 2^15 blocks (further on its host layout is different).
+    This exercises both key words, the low bits of counter word 2 and every
+    round; counter words 0, 1, 3 and the high bits of word 2 are compared
+    with cuRAND's device generator in the GPU suite."""
+    import ctypes
+    lib = _curand_host_lib()
+    if lib is None:
+        pytest.skip("cuRAND library not found")
+    PHILOX = 161  # CURAND_RNG_PSEUDO_PHILOX4_32_10
+    for seed, first_block, nblk in [(0, 0, 1 << 14), (0xF00DBEEF12345678, 0, 1024),
+                                    (0xFFFFFFFF00000001, 12345, 256),
+                                    (0x0123456789ABCDEF, (1 << 15) - 100, 100),
+                                    (0x8000000080000000, 1 << 14, 64)]:
+        gen = ctypes.c_void_p()
+        assert lib.curandCreateGeneratorHost(ctypes.byref(gen), PHILOX) == 0
+        try:
+            assert lib.curandSetPseudoRandomGeneratorSeed(gen, ctypes.c_ulonglong(seed)) == 0
+            assert lib.curandSetGeneratorOffset(gen, ctypes.c_ulonglong(4 * first_block)) == 0
+            ref = np.zeros(4 * nblk, np.uint32)
+            assert lib.curandGenerate(gen, ref.ctypes.data_as(ctypes.c_void_p),
+                                      ctypes.c_size_t(ref.size)) == 0
+        finally:
+            lib.curandDestroyGenerator(gen)
+        key = [seed & 0xFFFFFFFF, seed >> 32]
+        got = np.array([w for j in range(nblk)
+                        for w in orc.philox([0, 0, first_block + j, 0], key)], np.uint32)
+        assert np.array_equal(got, ref), (hex(seed), first_block)
+
+
 def test_uniform_counter_layout(orc):
     seed, cyc = 0x0123456789ABCDEF, 0x0000BEEF00C0FFEE
     for (b, pos, tag) in [(0, 0, 0), (5, 3, 1), (1 << 20, 31, 2)]:

@@ -27,10 +27,42 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes]
 
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};  // context the address belongs to
 
-// Device address of the array for the current device, looked up once per
-// device with that device current.  (In host code the array's name is only a
-// host-side stand-in, never a device address.)
+// Unique id of the calling thread's current context (0 if unavailable): the
+// array's address is valid for one context, and a device reset or a new
+// primary context loads the module again, possibly elsewhere.
+unsigned long long current_context_id() {
+  typedef CUresult (*GetCurrentFn)(CUcontext*);
+  typedef CUresult (*GetIdFn)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) == cudaSuccess &&
+        q1 == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) == cudaSuccess &&
+        q2 == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<GetCurrentFn>(f1);
+      get_id = reinterpret_cast<GetIdFn>(f2);
+    }
+    looked_up = true;
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx &&
+      get_id(ctx, &id) == CUDA_SUCCESS)
+    return id;
+  return 0;
+}
+
+// Device address of the array for the current device, looked up with that
+// device current the first time the device is used in a context (and again
+// if the context changed, e.g. after cudaDeviceReset).  In host code the
+// array's name is only a host-side stand-in, never a device address.
 void* scratch_for_current_device(spec_status* err) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
@@ -38,13 +70,15 @@ void* scratch_for_current_device(spec_status* err) {
     return nullptr;
   }
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
+  const unsigned long long ctx = current_context_id();
+  if (!g_scratch_addr[dev] || (ctx != 0 && ctx != g_scratch_ctx[dev])) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
       *err = SPEC_ERR_CUDA;
       return nullptr;
     }
     g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = current_context_id();
   }
   return g_scratch_addr[dev];
 }

@@ -154,7 +154,8 @@ spec_status spec_cycle(const spec_params *p, const void *base, const void *targe
  * every GPU that loads it until the process exits; nothing is allocated per
  * call.  Shapes whose spec_workspace_size exceeds 8 MiB are rejected with
  * SPEC_ERR_WORKSPACE (and a message on stderr).  The first call on a device
- * looks up the array's device address; make that first call before any stream
+ * looks up the array's device address (again after the device's context was
+ * replaced, e.g. by cudaDeviceReset); make that first call before any stream
  * capture.  All calls share the array: calls that overlap on the GPU race, so
  * order them on one stream.  status_out (device int32, may be NULL) receives
  * the device-side status of the call, stream-ordered after it. */

@@ -63,3 +63,36 @@ def test_recorded_traffic_only_for_the_profiled_source():
     p = os.path.join(ROOT, "profiles", "k_cycle_c3_ncu.json")
     d = json.load(open(p))
     assert bench.recorded_traffic(d["csrc_hash"]) == d["dram_bytes_per_launch"]
+
+
+def test_clock_sampler_short_region_takes_the_nearest_samples():
+    # a timed region shorter than the sampling period: the samples on each side
+    c = bench.ClockSampler(0)
+    row = lambda mhz: ["0", str(mhz), "1965", "300.0", "0x0", "Not Active", "Not Active",
+                       "Not Active", "Not Active"]
+    c.samples = [(1.0, row(1900)), (2.0, row(1965)), (3.0, row(1950)), (4.0, row(1000))]
+    c.t0, c.t1 = 2.2, 2.3
+    s = c.summary()
+    assert s["samples"] == 2 and s["sm_mhz"] == (1965 + 1950) / 2
+    assert "nearest" in s["window"]
+
+
+def test_w_l2_bytes_counts_the_streamed_chunks():
+    # V = 129280: 1010 chunks of 128 tokens, 7 per CTA on 148 SMs (145 CTAs, the
+    # last with 2); 3 chunks per CTA stay in tensor memory, the rest stream every
+    # MMA round (16 draft steps + the final step)
+    w = synth.WORKLOADS["c3"]
+    streamed = 144 * (7 - 3) + 0
+    assert bench.w_l2_bytes(w, 148) == streamed * 128 * 256 * 2 * 17
+    assert bench.w_l2_bytes(w, 148, greedy=True) == streamed * 128 * 256 * 2 * 16
+
+
+def test_near_threshold_counts_flagged_and_mismatched_rows():
+    K = 3
+    ref = {"tau": np.array([2, 4, 1]), "out": np.array([[5, 6, -1, -1], [1, 2, 3, 4], [9, -1, -1, -1]]),
+           "flag_draft": np.array([3, 3, 1]), "flag_accept": np.array([3, 3, 3]),
+           "flag_final": np.array([0, 0, 0])}
+    out = np.array([[5, 6, -1, -1], [1, 2, 3, 7], [8, -1, -1, -1]])
+    tau = np.array([2, 4, 1])
+    r = bench.near_threshold(ref, out, tau, K)
+    assert r == {"rows_checked": 3, "flagged": 1, "mismatched_unflagged": 1}

@@ -70,3 +70,28 @@ def test_no_alloc_rejects_shapes_beyond_its_buffer():
     fake = ctypes.c_void_p(0x1000)
     rc = sd.lib().spec_cycle_noalloc(ctypes.byref(p.c()), *([fake] * 10), None, None)
     assert rc == sd.SPEC_ERR_WORKSPACE
+
+
+def test_no_alloc_reports_a_device_error_and_the_next_call_starts_clean():
+    """A last token outside [0, V) is caught on the device (clamped, never used
+    as an address) and reported through status_out.  The shared array keeps
+    that call's status; the next call clears it first, and its outputs equal
+    spec_cycle's with a fresh workspace."""
+    w = synth.Workload("na", B=5, K=3, V=1000, r=64, dtype="bf16", sigma=0.6, seed=72, uw_std=0.3)
+    d = synth.make(w)
+    dd = {k: v.cuda() for k, v in d.items()}
+    p = sd.Params(B=w.B, K=w.K, V=w.V, r=w.r, dtype=w.dtype, temperature=1.0, seed=14, cycle=2)
+    bad = dd["last_token"].clone()
+    bad[1] = w.V + 7
+    o = sd.alloc_outputs(p)
+    status = torch.full((1,), -99, dtype=torch.int32, device="cuda")
+    sd.cycle_noalloc(p, dd["base"], dd["target"], dd["U"], dd["W"], bad, o["draft"], o["out"],
+                     o["tau"], o["p_draft"], o["q_draft"], status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == sd.SPEC_ERR_TOKEN_RANGE
+    ref = _with_workspace(p, dd)
+    got = _no_alloc(p, dd)
+    for k in ("draft", "out", "tau"):
+        assert np.array_equal(got[k], ref[k]), k
+    for k in ("p_draft", "q_draft"):
+        np.testing.assert_allclose(got[k], ref[k], rtol=0, atol=PROB_TOL, equal_nan=True)

@@ -170,6 +170,8 @@ size_t spec_workspace_size(const spec_params* p) {
   const char* why = nullptr;
   if (cycle_geometry(p->B, p->K, p->V, p->r, p->dtype, p->flags, sms, &g, &why))
     need = std::max(need, cycle_ws_bytes(p->K, g));
+  if (cycle_tc_geometry(p->B, p->K, p->V, p->r, p->dtype, p->flags, sms, &g, &why))
+    need = std::max(need, cycle_tc_ws_bytes(p->K, g));
   return round256(sizeof(WsHeader) + need);
 }
 
@@ -216,6 +218,48 @@ spec_status spec_markov_bias(const spec_params* p, const void* U, const void* W,
   return e == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
 }
 
+// The fused cycle on the tensor-core path (geometry already decided).
+static spec_status run_cycle_tc(const spec_params* p, const CycleGeom& g, const void* base,
+                                const void* target, const void* U, const void* W,
+                                const int32_t* last_token, int32_t* draft, int32_t* out,
+                                int32_t* tau, float* p_draft, float* q_draft, void* ws,
+                                spec_stream_t stream) {
+  CUtensorMap tmW;
+  if (!make_tmap_W(&tmW, W, p->r, p->V, kCycleWBoxK)) return SPEC_ERR_CUDA;
+  CycleLaunch L;
+  memset(&L, 0, sizeof(L));
+  L.base = base;
+  L.target = target;
+  L.U = U;
+  L.W = W;
+  L.last_token = last_token;
+  L.draft = draft;
+  L.out = out;
+  L.tau = tau;
+  L.p_draft = p_draft;
+  L.q_draft = q_draft;
+  L.B = p->B;
+  L.K = p->K;
+  L.V = p->V;
+  L.r = p->r;
+  L.dtype = p->dtype;
+  L.mode = MODE_CYCLE;
+  L.greedy = p->greedy ? 1 : 0;
+  L.temperature = p->temperature;
+  L.seed = p->seed;
+  L.cycle = p->cycle;
+  L.row0 = p->row_offset;
+  L.spin = spin_of(p);
+  L.trace = (p->flags & SPEC_FLAG_TRACE) != 0;
+  cudaError_t e = launch_cycle_tc(L, g, header_of(ws), body_of(ws), &tmW, (cudaStream_t)stream);
+  g_last_launches = 1;
+  if (e != cudaSuccess) {
+    fprintf(stderr, "specdec: launch failed: %s\n", cudaGetErrorString(e));
+    return SPEC_ERR_CUDA;
+  }
+  return SPEC_OK;
+}
+
 static spec_status run_cycle(const spec_params* p, int mode, const void* base, const void* target,
                              const void* U, const void* W, const int32_t* last_token,
                              int32_t* draft, int32_t* out, int32_t* tau, float* p_draft,
@@ -234,6 +278,9 @@ static spec_status run_cycle(const spec_params* p, int mode, const void* base, c
   if (sms <= 0) return SPEC_ERR_CUDA;
   CycleGeom g;
   const char* why = nullptr;
+  if (mode == MODE_CYCLE && cycle_tc_geometry(p->B, p->K, p->V, p->r, p->dtype, p->flags, sms, &g, &why))
+    return run_cycle_tc(p, g, base, target, U, W, last_token, draft, out, tau, p_draft, q_draft, ws,
+                        stream);
   if (!cycle_geometry(p->B, p->K, p->V, p->r, p->dtype, p->flags, sms, &g, &why)) {
     fprintf(stderr, "specdec: unsupported shape: %s\n", why);
     return SPEC_ERR_UNSUPPORTED;

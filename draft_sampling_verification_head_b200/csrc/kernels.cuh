@@ -80,6 +80,15 @@ struct CycleLaunch {
 cudaError_t launch_cycle(const CycleLaunch& L, const CycleGeom& g, WsHeader* hdr, uint8_t* body,
                          const CUtensorMap* tmW, const CUtensorMap* tmBase, cudaStream_t st);
 
+// Tensor-core path of the fused cycle (bf16, rank a multiple of 64 up to 256):
+// W^T partly resident in tensor memory, double-buffered accumulators, exact
+// bucket statistics.  Geometry returns false for other shapes.
+bool cycle_tc_geometry(int B, int K, int V, int r, int dtype, uint32_t flags, int num_sms,
+                       CycleGeom* g, const char** why);
+size_t cycle_tc_ws_bytes(int K, const CycleGeom& g);
+cudaError_t launch_cycle_tc(const CycleLaunch& L, const CycleGeom& g, WsHeader* hdr, uint8_t* body,
+                            const CUtensorMap* tmW, cudaStream_t st);
+
 // ---- Tensor maps --------------------------------------------------------------
 bool make_tmap_W(CUtensorMap* m, const void* W, int r, int V, int box_k);
 constexpr int kCycleWBoxK = 16;  // rank rows per W box of the fused cycle (one MMA K-step)

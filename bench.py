@@ -201,12 +201,15 @@ def cpu_baseline(w, d, max_seconds=20.0):
 
 
 def near_threshold(ref, out, tau, K):
-    """Rows of the oracle sample whose draws include a near-threshold decision
-    (counted, not compared), and unflagged rows whose emitted tokens or tau
-    differ from the oracle's (expected 0)."""
+    """Rows of the oracle sample whose outcome depends on a near-threshold
+    decision (a draft or accept decision flagged at or before the stop row, or
+    a flagged final draw: counted, not compared), and unflagged rows whose
+    emitted tokens or tau differ from the oracle's (expected 0)."""
     flagged = mism = 0
     for b in range(len(ref["tau"])):
-        if ref["flag_draft"][b] < K or ref["flag_accept"][b] < K or ref["flag_final"][b]:
+        stop = int(ref["tau"][b]) - 1
+        limit = min(int(ref["flag_draft"][b]), int(ref["flag_accept"][b]))
+        if limit <= min(stop, K - 1) or ref["flag_final"][b]:
             flagged += 1
         elif int(tau[b]) != int(ref["tau"][b]) or list(out[b]) != list(ref["out"][b]):
             mism += 1

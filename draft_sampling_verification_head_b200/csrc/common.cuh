@@ -28,7 +28,9 @@ struct WsHeader {
   uint32_t exit_count;  // CTAs that finished the current launch
   uint32_t abort;       // nonzero once a CTA of the current launch gave up
   uint32_t rec;         // row records published in the current launch
-  uint32_t pad[55];
+  uint32_t pad[54];
+  uint32_t events;      // tensor-core cycle: step events of all earlier launches on this
+                        // workspace (record tags); kept last so a reset of the rest keeps it
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
@@ -61,6 +63,14 @@ SPEC_DEV uint32_t ld_acquire_u32(const uint32_t* p) {
 }
 SPEC_DEV void red_release_add_u32(uint32_t* p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+SPEC_DEV uint64_t ld_acquire_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+SPEC_DEV void st_release_u64(uint64_t* p, uint64_t v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 SPEC_DEV uint32_t ld_volatile_u32(const uint32_t* p) {
   return *reinterpret_cast<const volatile uint32_t*>(p);

@@ -54,7 +54,7 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kTargetWarp0 = 10;     // warps 10 and 11: target row statistics
 constexpr int kThreads = 384;
-constexpr int kTS = 8;               // row-slice slots per target warp
+constexpr int kTSMax = 16;           // row-slice slots per target warp, at most
 constexpr int kNS = 6;               // W ring stages
 constexpr int kKS = 4;               // MMA K-steps (16 rank rows each) per stage
 constexpr int kWChunk = kCH * 16 * 2;         // 4 KB: one K-step of one chunk
@@ -84,6 +84,7 @@ struct ArgsTC {
   float2* tpart;     // [2][K+1][N][kMaxG]: target (max, sum) or (max, idx)
   int32_t* tokens;   // [2][K][N]
   RecT* rec;         // [2][K+1][N] row records (slot K: the final draw)
+  uint64_t* rtag;    // [2][K+1][N] record tags: (tag << 32) | accept << 31 | token
   float2* gbk;       // [G][nbk][N] bucket statistics of every CTA (current step)
   uint64_t* trace;   // [K+2][kTracePhases] device timeline of CTA 0, or null
   int B, K, V, r, G, nc, nchunks, greedy, ngroups, NT;
@@ -91,6 +92,7 @@ struct ArgsTC {
   uint64_t seed, cycle, spin;
   uint32_t row0;     // global index of batch row 0 (Philox counter word 1)
   int nbk;           // buckets per CTA (4 per chunk)
+  int nts;           // row-slice slots per target warp (what shared memory holds)
 };
 
 // One record per batch row and step, written by the row's reducer.
@@ -113,7 +115,7 @@ template <int N>
 struct CtlT {
   uint64_t wfull[kNS], wempty[kNS], dfull[2], dfree[2];
   uint64_t bready, tready, mmadone;
-  uint64_t tfull[2][kTS];  // target row slices landed (one ring per target warp)
+  uint64_t tfull[2][kTSMax];  // target row slices landed (one ring per target warp)
   uint64_t tgo, tdone;     // target job may start / has published its partials
   uint32_t tmem_slot;
   int32_t abort_local;
@@ -121,13 +123,14 @@ struct CtlT {
   int32_t alive[N];
   int32_t stoprow[N];
   int32_t tok[N];
+  int32_t acc[N];        // accept outcome of the step, from the record tags
   float zM[N], zS[N];    // draft statistics of the stop row
   float fMt[N], fSt[N];  // target statistics of the final row (stop row or row K)
   alignas(16) float4 fcst[N];  // final step: target max, 1 / target sum, draft max, 1 / draft sum
   float qa[4][N], qb[4][N];    // per-quadrant partials: draft / final residual
   RecT rrec[N];          // records of the rows this CTA reduces, before publication
   float zpart[8][32];    // per-warp partial Markov biases of a draw's 32 tokens
-  int32_t dbk;           // the draw's bucket inside the owner CTA
+  int32_t dbk;           // the draw's bucket (entry of the row's bucket array)
   float dtin;            // inverse-CDF target inside that bucket
 };
 
@@ -259,7 +262,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
   uint8_t* sU = sW + (size_t)kNS * kWStage;                 // nkb x N x 128 B
   float* sT = reinterpret_cast<float*>(sU + (size_t)nkb * N * 128);  // 8 x 32 x NCOL floats
   const size_t rslot = (size_t)a.nc * kCH * sizeof(__nv_bfloat16);  // one row slice of the CTA
-  uint8_t* sR = reinterpret_cast<uint8_t*>(sT + 8 * 32 * NCOL);      // 2 x kTS row slices
+  uint8_t* sR = reinterpret_cast<uint8_t*>(sT + 8 * 32 * NCOL);      // 2 x nts row slices
+  const int kTS = a.nts;
   CtlT<N>* ctl = reinterpret_cast<CtlT<N>*>(sR + 2 * kTS * rslot);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -291,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
     mbar_init(&ctl->tready, 1);
     mbar_init(&ctl->mmadone, 1);
     for (int w = 0; w < 2; ++w)
-      for (int i = 0; i < kTS; ++i) mbar_init(&ctl->tfull[w][i], 1);
+      for (int i = 0; i < kTSMax; ++i) mbar_init(&ctl->tfull[w][i], 1);
     mbar_init(&ctl->tgo, 1);
     mbar_init(&ctl->tdone, 2);
     ctl->abort_local = 0;
@@ -305,6 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t taddr = ctl->tmem_slot;
+  if (tid == 0) mbar_arrive(&ctl->tgo);  // the first target job needs nothing else: start it now
 
   // =========================================================================
   // W producer: first the NT resident chunks (read once, by the compute warps,
@@ -440,11 +445,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
           break;
         }
         const bool last = j == K - 1;
+        {  // the next job's target rows of this warp's rows into L2
+          const int nl2 = 2 * lane + tw;
+          if (j + 1 < K && nl2 < nb_g && nl2 < N &&
+              *reinterpret_cast<volatile int32_t*>(&ctl->alive[nl2]) != 0) {
+            const int64_t bb = (int64_t)g * N + nl2;
+            prefetch_l2_bulk(target + (bb * (K + 1) + j + 1) * V + vlo, bytes);
+            if (j + 2 == K) prefetch_l2_bulk(target + (bb * (K + 1) + K) * V + vlo, bytes);
+          }
+        }
         // rows n = 2 l + tw still verifying (a snapshot: a row that stops
         // meanwhile only costs an unused slice)
         const int nl = 2 * lane + tw;
-        const uint32_t rows = __ballot_sync(FULL, nl < nb_g && nl < N &&
-                                                      *reinterpret_cast<volatile int32_t*>(&ctl->alive[nl]) != 0);
+        const uint32_t rows = __ballot_sync(
+            FULL, nl < nb_g && nl < N &&
+                      (j == 0 || *reinterpret_cast<volatile int32_t*>(&ctl->alive[nl]) != 0));
         // items: (row, target row j) and, at the last job, (row, target row K)
         uint32_t imask = rows, cmask = rows;
         int isub = 0, csub = 0;
@@ -545,7 +560,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
     const int jj = lane / L, tg = lane % L;
     const int nrow = n0 + jj;              // the batch row this lane holds after the transpose
     float* tbuf = sT + warp * 32 * NCOL;
-    uint32_t cc = 0, nbar = 0, rec_expected = 0;
+    uint32_t cc = 0, nbar = 0;
+    const uint32_t ev0 = ld_volatile_u32(&hdr->events);  // record tags of this launch start here
     bool failed = false;
     auto soft_fail = [&](int code, int site, int x, int y) {
       record_error(hdr, code, site, x, y);
@@ -729,6 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         }
       }
       named_sync();
+      if (j == 0 && kind == 0) mark(g, i, 14);
       const int bk = ctl->dbk;
       const int v0 = (o * a.nc + (bk >> 2)) * kCH + (bk & 3) * 32;
       const int v = v0 + lane, vc = min(v, V - 1);
@@ -755,6 +772,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         ctl->zpart[warp][lane] = part;
       }
       named_sync();
+      if (j == 0 && kind == 0) mark(g, i, 15);
       if (warp == 0) {
         float bias = 0.f;
 #pragma unroll
@@ -960,18 +978,40 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
       // stochastic draws, one row at a time by the whole CTA
       if ((kind == 0 && !a.greedy) || kind == 2)
         for (int j = 0; j < mine; ++j) draw_row(kind, g, par, i, cta + j * G, j);
-      if (tid < mine)
-        store_rec(a.rec + ((int64_t)par * (K + 1) + slot) * N + (cta + tid * G), ctl->rrec[tid]);
+      if (tid < mine) {  // the record, then its tag (release: the record is visible first)
+        const int n = cta + tid * G;
+        const RecT& rc = ctl->rrec[tid];
+        const size_t at = ((size_t)par * (K + 1) + slot) * N + n;
+        store_rec(a.rec + at, rc);
+        const uint32_t tag = ev0 + (uint32_t)(g * (K + 1) + slot + 1);
+        st_release_u64(a.rtag + at, ((uint64_t)tag << 32) | ((uint64_t)(rc.acc & 1) << 31) |
+                                        (uint64_t)(uint32_t)(rc.token & 0x7fffffff));
+      }
       return mine;
     };
-    // publish this CTA's records and wait until every row's record exists
-    auto records_hop = [&](int mine, int nb_g) {
-      named_sync();
-      if (tid == 0) {
-        if (mine) red_release_add_u32(&hdr->rec, (uint32_t)mine);
-        rec_expected += (uint32_t)nb_g;
-        if (!grid_wait_count(hdr, &hdr->rec, rec_expected, a.spin, SITE_REC_WAIT))
+    // Wait until every row's record of this slot carries this step's tag;
+    // thread n < nb_g polls row n.  Returns false if the launch is aborted.
+    auto records_hop = [&](int g, int par, int slot, int nb_g) {
+      if (tid < nb_g) {
+        const uint64_t* t = a.rtag + ((size_t)par * (K + 1) + slot) * N + tid;
+        const uint32_t want = ev0 + (uint32_t)(g * (K + 1) + slot + 1);
+        bool ok = false;
+        for (uint64_t it = 0; it < a.spin; ++it) {
+          const uint64_t wv = ld_acquire_u64(t);
+          if ((uint32_t)(wv >> 32) == want) {
+            ok = true;
+            ctl->tok[tid] = (int32_t)(wv & 0x7fffffffu);
+            ctl->acc[tid] = (int32_t)((wv >> 31) & 1u);
+            break;
+          }
+          if ((it & 15) == 15 && ld_volatile_u32(&hdr->abort)) break;
+          __nanosleep(32);
+        }
+        if (!ok) {
+          if (!ld_volatile_u32(&hdr->abort))
+            record_error(hdr, SPEC_ERR_TIMEOUT, SITE_REC_WAIT, cta, 6000 + slot);
           ctl->abort_local = 1;
+        }
       }
       named_sync();
       return ctl->abort_local == 0;
@@ -999,11 +1039,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
           if (a.q_draft && a.greedy) a.q_draft[o] = NaNf;
         }
       }
-      // step 0's base logits of this CTA's slice into L2
-      if (tid < nb_g)
-        prefetch_l2_bulk(base + ((int64_t)g * N + tid) * K * V + vslice_lo, slice_bytes);
+      // step 0's base and target logits of this CTA's slice into L2
+      if (tid < nb_g) {
+        const int64_t b = (int64_t)g * N + tid;
+        prefetch_l2_bulk(base + b * K * V + vslice_lo, slice_bytes);
+        prefetch_l2_bulk(target + b * (K + 1) * V + vslice_lo, slice_bytes);
+        if (K == 1) prefetch_l2_bulk(target + (b * (K + 1) + 1) * V + vslice_lo, slice_bytes);
+      }
       named_sync();
-      if (tid == 0) mbar_arrive(&ctl->tgo);  // the target warps may take row 0 of this group
+      if (tid == 0 && g > 0) mbar_arrive(&ctl->tgo);  // the target warps may take row 0 of this group
       mark(g, K + 1, 0);
 
       for (int i = 0; i < K; ++i) {
@@ -1141,23 +1185,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         if (a.trace && g == 0 && tid == 0 && mine)
           atomicMax(reinterpret_cast<unsigned long long*>(a.trace) + (size_t)i * kTracePhases + 7,
                     (unsigned long long)globaltimer_ns());
-        if (!records_hop(mine, nb_g)) {
+        if (!records_hop(g, par, i, nb_g)) {
           failed = true;
           break;
         }
-        // the step's tokens, accept outcomes and statistics, from the records
+        // accept outcomes from the tags; a row that stops (or the bonus at the
+        // last step) reads its full record for the final step's statistics
         for (int n = tid; n < nb_g; n += kComputeThreads) {
-          const RecT r = load_rec(a.rec + ((int64_t)par * (K + 1) + i) * N + n);
-          ctl->tok[n] = r.token;
-          if (ctl->alive[n]) {
-            if (!r.acc) {
+          if (ctl->alive[n] && (!ctl->acc[n] || last)) {
+            const RecT r = load_rec(a.rec + ((int64_t)par * (K + 1) + i) * N + n);
+            if (!ctl->acc[n]) {
               ctl->alive[n] = 0;
               ctl->stoprow[n] = i;
               ctl->zM[n] = r.M;    // draft statistics of the stop row
               ctl->zS[n] = r.S;
               ctl->fMt[n] = r.Mt;  // target statistics of the stop row
               ctl->fSt[n] = r.St;
-            } else if (last) {
+            } else {
               ctl->fMt[n] = r.MtK;  // every draft accepted: the bonus comes from row K
               ctl->fSt[n] = r.StK;
             }
@@ -1278,8 +1322,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         }
         mark(g, K, 4);
         // the reducers draw each row's residual / bonus token and write it
-        const int mine = reduce_rows(2, g, par, K, nb_g);
-        if (!records_hop(mine, nb_g)) {
+        reduce_rows(2, g, par, K, nb_g);
+        // the next group overwrites the bucket statistics: every draw is done first
+        if (g + 1 < a.ngroups && !records_hop(g, par, K, nb_g)) {
           failed = true;
           break;
         }
@@ -1319,22 +1364,36 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
       hdr->bar = 0;
       hdr->rec = 0;
       hdr->abort = 0;
+      hdr->events += (uint32_t)(a.ngroups * (K + 1));  // tags of the next launch differ
       __threadfence();
       atomicExch(&hdr->exit_count, 0u);
     }
   }
 }
 
+constexpr size_t kSmemBudget = 227 * 1024;
+
+// Shared memory without the target rings, and the ring slots that fit beside it.
 template <int N>
-size_t smem_bytes_tc(int r, int nc) {
+size_t smem_fixed_tc(int r) {
   constexpr int NCOL = N / 2;
   size_t s = 1024;  // alignment slack
   s += (size_t)kNS * kWStage;
   s += (size_t)(r / 64) * N * 128;
   s += (size_t)8 * 32 * NCOL * sizeof(float);
-  s += (size_t)2 * kTS * nc * kCH * sizeof(__nv_bfloat16);
   s += sizeof(CtlT<N>);
   return s;
+}
+template <int N>
+int ring_slots_tc(int r, int nc) {
+  const size_t fixed = smem_fixed_tc<N>(r);
+  const size_t rslot = (size_t)nc * kCH * sizeof(__nv_bfloat16);
+  if (fixed + 2 * rslot > kSmemBudget) return 0;
+  return (int)std::min<size_t>(kTSMax, (kSmemBudget - fixed) / (2 * rslot));
+}
+template <int N>
+size_t smem_bytes_tc(int r, int nc) {
+  return smem_fixed_tc<N>(r) + (size_t)2 * ring_slots_tc<N>(r, nc) * nc * kCH * sizeof(__nv_bfloat16);
 }
 
 template <int N>
@@ -1352,6 +1411,7 @@ size_t dpart_bytes(int K, int N) { return a256(sizeof(float4) * 2 * (size_t)(K +
 size_t tpart_bytes(int K, int N) { return a256(sizeof(float2) * 2 * (size_t)(K + 1) * N * kMaxG); }
 size_t tok_bytes(int K, int N) { return a256(sizeof(int32_t) * 2 * (size_t)K * N); }
 size_t rec_bytes(int K, int N) { return a256(sizeof(RecT) * 2 * (size_t)(K + 1) * N); }
+size_t rtag_bytes(int K, int N) { return a256(sizeof(uint64_t) * 2 * (size_t)(K + 1) * N); }
 size_t gbk_bytes(const CycleGeom& g) { return a256(sizeof(float2) * (size_t)g.G * g.nc * 4 * g.N); }
 
 }  // namespace
@@ -1375,7 +1435,9 @@ bool cycle_tc_geometry(int B, int K, int V, int r, int dtype, uint32_t flags, in
   g->tc = true;
   g->smem = g->N == 64 ? smem_bytes_tc<64>(r, nc)
                         : (g->N == 32 ? smem_bytes_tc<32>(r, nc) : smem_bytes_tc<16>(r, nc));
-  if (g->smem > 227 * 1024) {
+  const int nts = g->N == 64 ? ring_slots_tc<64>(r, nc)
+                             : (g->N == 32 ? ring_slots_tc<32>(r, nc) : ring_slots_tc<16>(r, nc));
+  if (nts < 2 || g->smem > kSmemBudget) {
     *why = "shared memory budget exceeded";
     return false;
   }
@@ -1385,7 +1447,7 @@ bool cycle_tc_geometry(int B, int K, int V, int r, int dtype, uint32_t flags, in
 
 size_t cycle_tc_ws_bytes(int K, const CycleGeom& g) {
   return cycle_trace_bytes(K) + dpart_bytes(K, g.N) + tpart_bytes(K, g.N) + tok_bytes(K, g.N) +
-         rec_bytes(K, g.N) + gbk_bytes(g);
+         rec_bytes(K, g.N) + rtag_bytes(K, g.N) + gbk_bytes(g);
 }
 
 cudaError_t launch_cycle_tc(const CycleLaunch& L, const CycleGeom& g, WsHeader* hdr, uint8_t* body,
@@ -1414,8 +1476,12 @@ cudaError_t launch_cycle_tc(const CycleLaunch& L, const CycleGeom& g, WsHeader* 
   body += tok_bytes(L.K, g.N);
   a.rec = reinterpret_cast<RecT*>(body);
   body += rec_bytes(L.K, g.N);
+  a.rtag = reinterpret_cast<uint64_t*>(body);
+  body += rtag_bytes(L.K, g.N);
   a.gbk = reinterpret_cast<float2*>(body);
   a.nbk = g.nc * 4;
+  a.nts = g.N == 64 ? ring_slots_tc<64>(L.r, g.nc)
+                    : (g.N == 32 ? ring_slots_tc<32>(L.r, g.nc) : ring_slots_tc<16>(L.r, g.nc));
   a.B = L.B;
   a.K = L.K;
   a.V = L.V;

@@ -104,8 +104,12 @@ extern "C" spec_status spec_cycle_noalloc(const spec_params* p, const void* base
   void* ws = scratch_for_current_device(&err);
   if (!ws) return err;
   cudaStream_t st = (cudaStream_t)stream;
-  // the previous call leaves its status and counters behind: start from zero
-  if (cudaMemsetAsync(ws, 0, sizeof(specdec::WsHeader), st) != cudaSuccess) return SPEC_ERR_CUDA;
+  // the previous call leaves its status and counters behind: start from zero.
+  // The header's last word (the count of earlier step events, which keeps the
+  // record tags of consecutive calls apart) is kept; the rest of the scratch
+  // needs no clearing: a launch writes every entry before reading it.
+  if (cudaMemsetAsync(ws, 0, sizeof(specdec::WsHeader) - sizeof(uint32_t), st) != cudaSuccess)
+    return SPEC_ERR_CUDA;
   const spec_status s = spec_cycle(p, base, target, U, W, last_token, draft, out, tau, p_draft,
                                    q_draft, ws, stream);
   if (s != SPEC_OK) return s;

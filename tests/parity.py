@@ -12,6 +12,14 @@ import numpy as np
 
 PROB_TOL = 1e-5
 
+# (case, cycle, rows compared, rows with a near-threshold decision): filled by
+# the GPU tests, printed in the test session's terminal summary
+NEAR_THRESHOLD = []
+
+
+def note_near(case: str, cycle: int, rows: int, flagged: int):
+    NEAR_THRESHOLD.append((case, cycle, rows, flagged))
+
 
 def compare_cycle(gpu: dict, orc: dict, K: int, rows=None, check_probs=True):
     """gpu/orc: dicts of numpy arrays (draft, out, tau, p_draft, q_draft) for the

@@ -89,8 +89,10 @@ def test_w_l2_bytes_counts_the_streamed_chunks():
 
 def test_near_threshold_counts_flagged_and_mismatched_rows():
     K = 3
+    # row 0: a draft flag after its stop row (position 2 > stop 1) does not count;
+    # row 1: all accepted, last token differs (mismatch); row 2: flagged at the stop row
     ref = {"tau": np.array([2, 4, 1]), "out": np.array([[5, 6, -1, -1], [1, 2, 3, 4], [9, -1, -1, -1]]),
-           "flag_draft": np.array([3, 3, 1]), "flag_accept": np.array([3, 3, 3]),
+           "flag_draft": np.array([2, 3, 0]), "flag_accept": np.array([3, 3, 3]),
            "flag_final": np.array([0, 0, 0])}
     out = np.array([[5, 6, -1, -1], [1, 2, 3, 7], [8, -1, -1, -1]])
     tau = np.array([2, 4, 1])

@@ -42,7 +42,8 @@ class _Params(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("K", ctypes.c_int32), ("V", ctypes.c_int32),
                 ("r", ctypes.c_int32), ("dtype", ctypes.c_int32), ("draft_dtype", ctypes.c_int32),
                 ("temperature", ctypes.c_double), ("greedy", ctypes.c_int32),
-                ("seed", ctypes.c_uint64), ("cycle", ctypes.c_uint64)]
+                ("seed", ctypes.c_uint64), ("cycle", ctypes.c_uint64),
+                ("verify_len", ctypes.c_void_p)]
 
 
 class _Outputs(ctypes.Structure):
@@ -94,13 +95,19 @@ class Params:
     seed: int = 0
     cycle: int = 0
     draft_dtype: str | None = None  # verify-only: dtype of the given draft logits
+    verify_len: np.ndarray | None = None  # [B] int32 per-row verify length K_b (1..K), or None
 
     def c(self) -> _Params:
         dd = self.draft_dtype or self.dtype
         # the temperature is the fp32 value the GPU receives, widened exactly
         T = float(np.float32(self.temperature))
+        vl = None
+        if self.verify_len is not None:
+            self._vl = np.ascontiguousarray(self.verify_len, dtype=np.int32)  # kept alive
+            vl = self._vl.ctypes.data_as(ctypes.c_void_p)
         return _Params(self.B, self.K, self.V, self.r, _DT[self.dtype], _DT[dd], T,
-                       1 if self.greedy else 0, self.seed & (2**64 - 1), self.cycle & (2**64 - 1))
+                       1 if self.greedy else 0, self.seed & (2**64 - 1), self.cycle & (2**64 - 1),
+                       vl)
 
 
 def _raw(a: np.ndarray, dtype: str) -> np.ndarray:

@@ -40,14 +40,18 @@ def draft_q(base, U, W, i, prev, T):
     return softmax(z, T)
 
 
-def exact_law(base, target, U, W, last_token, T, rule="standard"):
+def exact_law(base, target, U, W, last_token, T, rule="standard", verify_len=None):
     """Return {(tau, out_tuple): probability} for one batch row.
 
     base: [K, V], target: [K+1, V], U: [V, r], W: [r, V] (float64-convertible).
+    verify_len: the row's verify length K_b (1..K; default K): positions
+    0..K_b-1 are drafted and verified, the bonus comes from target row K_b.
     """
     base = np.asarray(base, np.float64)
     target = np.asarray(target, np.float64)
     K, V = base.shape
+    if verify_len is not None:
+        K = int(verify_len)
     P = [softmax(target[i], T) for i in range(K + 1)]
     law = defaultdict(float)
 

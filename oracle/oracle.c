@@ -213,17 +213,29 @@ static int check_params(const orc_params *P, int32_t b_begin, int32_t b_end) {
   if (!P || P->B < 0 || P->K < 1 || P->V < 1 || P->r < 0) return -1;
   if (b_begin < 0 || b_end > P->B || b_begin > b_end) return -1;
   if (!P->greedy && !(P->temperature > 0.0)) return -1;
+  if (P->verify_len)
+    for (int32_t b = b_begin; b < b_end; ++b)
+      if (P->verify_len[b] < 1 || P->verify_len[b] > P->K) return -4;
   return 0;
+}
+
+/* Verify length of row b: K_b, or K without a per-row array. */
+static int32_t verify_len_of(const orc_params *P, int32_t b) {
+  return P->verify_len ? P->verify_len[b] : P->K;
 }
 
 /* Draft one row: fills d[K], qd[K], zrows[K*V] (z values), flag. */
 static int draft_row(const orc_params *P, const void *base, const void *U, const void *W,
                      int32_t b, int32_t prev0, int32_t *d, double *qd, double *zrows,
                      int32_t *flag_draft, double *scratch) {
-  const int32_t K = P->K, V = P->V;
+  const int32_t K = P->K, V = P->V, Kb = verify_len_of(P, b);
   int32_t prev = prev0;
   if (flag_draft) *flag_draft = K;
-  for (int32_t i = 0; i < K; ++i) {
+  for (int32_t i = Kb; i < K; ++i) {  /* positions past the verify length are not drafted */
+    d[i] = -1;
+    qd[i] = NAN;
+  }
+  for (int32_t i = 0; i < Kb; ++i) {
     double *z = zrows + (size_t)i * V;
     biased_row(P, base, U, W, b, i, prev, z);
     int32_t near = 0, tok;
@@ -253,12 +265,18 @@ static int draft_row(const orc_params *P, const void *base, const void *U, const
 static void verify_row(const orc_params *P, const void *target, const double *zrows,
                        const int32_t *d, int32_t b, int32_t *out, int32_t *tau, double *pd,
                        double *qd_out, int32_t *flag_accept, int32_t *flag_final) {
-  const int32_t K = P->K, V = P->V;
+  const int32_t Kfull = P->K, V = P->V;
+  const int32_t K = verify_len_of(P, b);  /* the row's verify length K_b; bonus from row K_b */
   const double T = P->temperature;
+  for (int32_t j = 0; j <= Kfull; ++j) out[j] = -1;
+  if (pd)
+    for (int32_t j = 0; j < Kfull; ++j) pd[j] = NAN;
+  if (qd_out)
+    for (int32_t j = 0; j < Kfull; ++j) qd_out[j] = NAN;
   double *trow = (double *)malloc(sizeof(double) * (size_t)V * (K + 1));
   for (int32_t i = 0; i <= K; ++i)
     for (int32_t v = 0; v < V; ++v)
-      trow[(size_t)i * V + v] = load_elem(target, P->dtype, ((int64_t)b * (K + 1) + i) * V + v);
+      trow[(size_t)i * V + v] = load_elem(target, P->dtype, ((int64_t)b * (Kfull + 1) + i) * V + v);
   if (P->greedy) {
     /* accept while argmax(target_i) == d_i; emit the target arg-max at the stop */
     int32_t i;
@@ -275,9 +293,7 @@ static void verify_row(const orc_params *P, const void *target, const double *zr
     }
     if (i == K) out[K] = argmax_lowest(trow + (size_t)K * V, V, NULL, 0.0);
     *tau = i + 1;
-    if (qd_out)
-      for (int32_t j = 0; j < K; ++j) qd_out[j] = NAN;
-    if (flag_accept) *flag_accept = K;
+    if (flag_accept) *flag_accept = Kfull;
     if (flag_final) *flag_final = 0;
     free(trow);
     return;
@@ -293,6 +309,7 @@ static void verify_row(const orc_params *P, const void *target, const double *zr
   for (int32_t i = 0; i <= K; ++i)
     u_res[i] = orc_uniform(P->seed, P->cycle, (uint32_t)b, (uint32_t)i, ORC_TAG_RESAMPLE);
   orc_verify_probs(K, V, p, q, d, u_acc, u_res, out, tau, pd, flag_accept, flag_final);
+  if (flag_accept && *flag_accept == K) *flag_accept = Kfull;  /* "no flag" is K */
   if (qd_out)
     for (int32_t i = 0; i < K; ++i) qd_out[i] = q[(size_t)i * V + d[i]];
   free(u_acc);
@@ -385,7 +402,7 @@ int orc_verify(const orc_params *P, const void *target, const void *draft_logits
   if (check_params(P, b_begin, b_end) || !target || !draft_logits || !draft || !o) return -1;
   const int32_t K = P->K, V = P->V;
   for (int32_t b = b_begin; b < b_end; ++b)
-    for (int32_t i = 0; i < K; ++i)
+    for (int32_t i = 0; i < verify_len_of(P, b); ++i)
       if (draft[(size_t)b * K + i] < 0 || draft[(size_t)b * K + i] >= V) return -2;
   int threads = 1;
 #pragma omp parallel

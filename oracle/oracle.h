@@ -66,6 +66,12 @@ typedef struct {
   int32_t greedy;
   uint64_t seed;
   uint64_t cycle;
+  /* [B] per-row verify length K_b in 1..K, or NULL (every row K).  aigest.pl
+   * "Optymalizacja weryfikacji i wydajności": a scheduler fixes the verify
+   * length of each request.  Reading: row b drafts and verifies positions
+   * 0..K_b-1 only and takes its bonus from target row K_b (the rule above
+   * with K_b in place of K); draft[b, i] = -1 and q_draft NaN for i >= K_b. */
+  const int32_t *verify_len;
 } orc_params;
 
 /* Per-row outputs for rows [b_begin, b_end); arrays are indexed by b - b_begin.

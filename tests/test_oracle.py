@@ -315,6 +315,102 @@ def test_planted_oracle_mistakes_are_rejected(orc, tmp_path, plant):
     assert min(pv) < 1e-6, pv
 
 
+# ----------------------------------------------------------------------------- per-row verify length K_b
+
+# aigest.pl "DeepSeek prezentuje DSpark", "Optymalizacja weryfikacji i
+# wydajności": a scheduler fixes the verify length of each request and its early
+# stop keeps the method lossless.  Row b drafts and verifies positions
+# 0..K_b-1 and takes the bonus from target row K_b.
+
+@pytest.mark.parametrize("kb", [1, 2])
+@pytest.mark.parametrize("seed", [3, 9])
+def test_verify_length_lossless_by_enumeration(seed, kb):
+    w, d = _tiny_inputs(seed)
+    base, target = synth.as_float64(d["base"])[0], synth.as_float64(d["target"])[0]
+    U, W = synth.as_float64(d["U"]), synth.as_float64(d["W"])
+    law = EL.exact_law(base, target, U, W, int(d["last_token"][0]), 1.0, verify_len=kb)
+    assert abs(sum(law.values()) - 1.0) < 1e-12
+    assert max(t for t, _ in law) == kb + 1  # never more than K_b + 1 tokens
+    P = [EL.softmax(target[i], 1.0) for i in range(w.K + 1)]
+    for (i, prefix), (mass, dist) in EL.conditional_marginals(law, kb).items():
+        for v in range(w.V):
+            assert abs(dist.get(v, 0.0) - P[i][v]) < 1e-12, (i, prefix, v)
+
+
+def test_oracle_verify_length_samples_match_exact_law(orc):
+    """Oracle draws with K_b = 2 of K = 3 against the enumerated law (chi-square
+    on the first token and the tau histogram)."""
+    n, kb = 200_000, 2
+    w, d = _tiny_inputs(5)
+    base, target, last = _replicated(d, n)
+    P = orc.Params(B=n, K=w.K, V=w.V, r=w.r, dtype="f32", temperature=1.0, seed=42, cycle=3,
+                   verify_len=np.full(n, kb, np.int32))
+    o = orc.cycle(P, synth.to_numpy_raw(base), synth.to_numpy_raw(target),
+                  synth.to_numpy_raw(d["U"]), synth.to_numpy_raw(d["W"]), last.numpy())
+    law = EL.exact_law(synth.as_float64(d["base"])[0], synth.as_float64(d["target"])[0],
+                       synth.as_float64(d["U"]), synth.as_float64(d["W"]), int(last[0]), 1.0,
+                       verify_len=kb)
+    first, _, taus = EL.cell_probs(law, kb, w.V)
+    out, tau = o["out"], o["tau"]
+    assert tau.max() <= kb + 1 and np.all(out[:, kb + 1:] == -1)
+    assert np.all(o["draft"][:, kb:] == -1)
+    pv = [_pooled_chisq(np.bincount(out[:, 0], minlength=w.V), first, n),
+          _pooled_chisq(np.bincount(tau - 1, minlength=kb + 1), taus, n)]
+    assert min(pv) > 1e-3, pv
+
+
+@pytest.mark.parametrize("greedy", [False, True])
+def test_verify_length_k_equals_plain_cycle(orc, greedy):
+    w = synth.Workload("kbk", B=12, K=5, V=300, r=16, dtype="f32", sigma=0.6, seed=81, uw_std=0.3)
+    d = synth.make(w)
+    raw = [synth.to_numpy_raw(d[k]) for k in ("base", "target", "U", "W")]
+    kw = dict(B=w.B, K=w.K, V=w.V, r=w.r, dtype="f32", temperature=0.9, greedy=greedy, seed=7,
+              cycle=2)
+    a = orc.cycle(orc.Params(**kw), *raw, d["last_token"].numpy())
+    b = orc.cycle(orc.Params(**kw, verify_len=np.full(w.B, w.K, np.int32)), *raw,
+                  d["last_token"].numpy())
+    for k in ("draft", "out", "tau", "flag_draft", "flag_accept", "flag_final"):
+        assert np.array_equal(a[k], b[k]), k
+    np.testing.assert_array_equal(a["p_draft"], b["p_draft"])
+
+
+@pytest.mark.parametrize("greedy", [False, True])
+def test_verify_length_is_a_prefix_of_the_full_block(orc, greedy):
+    """The draws of a K_b row are the full block's first K_b draws (same random
+    counters): a row that stops before K_b emits exactly what the full block
+    emits; a row that accepts all K_b drafts emits them and a bonus drawn from
+    target row K_b."""
+    w = synth.Workload("kbp", B=64, K=6, V=400, r=16, dtype="f32", sigma=0.4, seed=82, uw_std=0.3)
+    d = synth.make(w)
+    raw = [synth.to_numpy_raw(d[k]) for k in ("base", "target", "U", "W")]
+    kb = (np.arange(w.B) % w.K + 1).astype(np.int32)
+    kw = dict(B=w.B, K=w.K, V=w.V, r=w.r, dtype="f32", temperature=1.0, greedy=greedy, seed=11,
+              cycle=4)
+    full = orc.cycle(orc.Params(**kw), *raw, d["last_token"].numpy())
+    part = orc.cycle(orc.Params(**kw, verify_len=kb), *raw, d["last_token"].numpy())
+    target = synth.as_float64(d["target"])
+    bonus_rows = 0
+    for b in range(w.B):
+        k = int(kb[b])
+        assert np.array_equal(part["draft"][b, :k], full["draft"][b, :k])
+        assert np.all(part["draft"][b, k:] == -1)
+        assert 1 <= part["tau"][b] <= k + 1 and np.all(part["out"][b, part["tau"][b]:] == -1)
+        if full["tau"][b] <= k:  # stopped inside the verified prefix: the same outcome
+            assert part["tau"][b] == full["tau"][b]
+            assert np.array_equal(part["out"][b], full["out"][b])
+        else:                    # every verified draft accepted: bonus from row K_b
+            bonus_rows += 1
+            assert part["tau"][b] == k + 1
+            assert np.array_equal(part["out"][b, :k], full["draft"][b, :k])
+            if greedy:
+                assert part["out"][b, k] == int(np.argmax(target[b, k]))
+            else:
+                p = EL.softmax(target[b, k], 1.0)
+                u = orc.uniform(11, 4, b, k, orc.TAG_RESAMPLE)
+                assert part["out"][b, k] == int(np.searchsorted(np.cumsum(p), u, side="right"))
+    assert bonus_rows > 5
+
+
 # ----------------------------------------------------------------------------- special cases (P4) and invariants (P5)
 
 def test_markov_off_draft_is_plain_categorical(orc):

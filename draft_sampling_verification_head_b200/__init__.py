@@ -29,6 +29,7 @@ _SIGS = {
     "spec_markov_bias_sample": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_verify_block": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_cycle": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "spec_cycle_kb": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_sync_status": (ctypes.c_int, [_P, _P]),
     "spec_cycle_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_l2_persist": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
@@ -163,6 +164,15 @@ def cycle(p: Params, base, target, U, W, last_token, draft, out, tau, p_draft, q
     _check(lib().spec_cycle(ctypes.byref(p.c()), _ptr(base), _ptr(target), _ptr(U), _ptr(W),
                             _ptr(last_token), _ptr(draft), _ptr(out), _ptr(tau), _ptr(p_draft),
                             _ptr(q_draft), _ptr(ws), _stream(stream)), "spec_cycle")
+
+
+def cycle_kb(p: Params, base, target, U, W, last_token, verify_len, draft, out, tau, p_draft,
+             q_draft, ws, stream=None):
+    """spec_cycle_kb: one cycle with a verify length K_b per row (int32 [B], 1..K)."""
+    _check(lib().spec_cycle_kb(ctypes.byref(p.c()), _ptr(base), _ptr(target), _ptr(U), _ptr(W),
+                               _ptr(last_token), _ptr(verify_len), _ptr(draft), _ptr(out),
+                               _ptr(tau), _ptr(p_draft), _ptr(q_draft), _ptr(ws),
+                               _stream(stream)), "spec_cycle_kb")
 
 
 def cycle_noalloc(p: Params, base, target, U, W, last_token, draft, out, tau, p_draft, q_draft,

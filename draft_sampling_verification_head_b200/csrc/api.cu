@@ -221,9 +221,9 @@ spec_status spec_markov_bias(const spec_params* p, const void* U, const void* W,
 // The fused cycle on the tensor-core path (geometry already decided).
 static spec_status run_cycle_tc(const spec_params* p, const CycleGeom& g, const void* base,
                                 const void* target, const void* U, const void* W,
-                                const int32_t* last_token, int32_t* draft, int32_t* out,
-                                int32_t* tau, float* p_draft, float* q_draft, void* ws,
-                                spec_stream_t stream) {
+                                const int32_t* last_token, const int32_t* vlen, int32_t* draft,
+                                int32_t* out, int32_t* tau, float* p_draft, float* q_draft,
+                                void* ws, spec_stream_t stream) {
   CUtensorMap tmW;
   if (!make_tmap_W(&tmW, W, p->r, p->V, kCycleWBoxK)) return SPEC_ERR_CUDA;
   CycleLaunch L;
@@ -233,6 +233,7 @@ static spec_status run_cycle_tc(const spec_params* p, const CycleGeom& g, const 
   L.U = U;
   L.W = W;
   L.last_token = last_token;
+  L.vlen = vlen;
   L.draft = draft;
   L.out = out;
   L.tau = tau;
@@ -262,8 +263,9 @@ static spec_status run_cycle_tc(const spec_params* p, const CycleGeom& g, const 
 
 static spec_status run_cycle(const spec_params* p, int mode, const void* base, const void* target,
                              const void* U, const void* W, const int32_t* last_token,
-                             int32_t* draft, int32_t* out, int32_t* tau, float* p_draft,
-                             float* q_draft, float* biased_out, void* ws, spec_stream_t stream) {
+                             const int32_t* vlen, int32_t* draft, int32_t* out, int32_t* tau,
+                             float* p_draft, float* q_draft, float* biased_out, void* ws,
+                             spec_stream_t stream) {
   g_last_launches = 0;
   spec_status s = check_params(p);
   if (s != SPEC_OK) return s;
@@ -279,8 +281,13 @@ static spec_status run_cycle(const spec_params* p, int mode, const void* base, c
   CycleGeom g;
   const char* why = nullptr;
   if (mode == MODE_CYCLE && cycle_tc_geometry(p->B, p->K, p->V, p->r, p->dtype, p->flags, sms, &g, &why))
-    return run_cycle_tc(p, g, base, target, U, W, last_token, draft, out, tau, p_draft, q_draft, ws,
-                        stream);
+    return run_cycle_tc(p, g, base, target, U, W, last_token, vlen, draft, out, tau, p_draft,
+                        q_draft, ws, stream);
+  if (vlen) {
+    fprintf(stderr, "specdec: per-row verify lengths need the tensor-core cycle (bf16, rank a "
+                    "multiple of 64 up to 256): %s\n", why);
+    return SPEC_ERR_UNSUPPORTED;
+  }
   if (!cycle_geometry(p->B, p->K, p->V, p->r, p->dtype, p->flags, sms, &g, &why)) {
     fprintf(stderr, "specdec: unsupported shape: %s\n", why);
     return SPEC_ERR_UNSUPPORTED;
@@ -290,6 +297,7 @@ static spec_status run_cycle(const spec_params* p, int mode, const void* base, c
   if (g.tc && !make_tmap_W(&tmW, W, p->r, p->V, kCycleWBoxK)) return SPEC_ERR_CUDA;
   if (!make_tmap_base(&tmBase, base, p->dtype, p->B, p->K, p->V, g.N, g.tc)) return SPEC_ERR_CUDA;
   CycleLaunch L;
+  memset(&L, 0, sizeof(L));
   L.base = base;
   L.target = target;
   L.U = U;
@@ -328,16 +336,25 @@ spec_status spec_markov_bias_sample(const spec_params* p, const void* base, cons
                                     const void* W, const int32_t* last_token, int32_t* draft,
                                     float* q_draft, float* biased_out, void* ws,
                                     spec_stream_t stream) {
-  return run_cycle(p, MODE_DRAFT, base, nullptr, U, W, last_token, draft, nullptr, nullptr,
-                   nullptr, q_draft, biased_out, ws, stream);
+  return run_cycle(p, MODE_DRAFT, base, nullptr, U, W, last_token, nullptr, draft, nullptr,
+                   nullptr, nullptr, q_draft, biased_out, ws, stream);
 }
 
 spec_status spec_cycle(const spec_params* p, const void* base, const void* target, const void* U,
                        const void* W, const int32_t* last_token, int32_t* draft, int32_t* out,
                        int32_t* tau, float* p_draft, float* q_draft, void* ws,
                        spec_stream_t stream) {
-  return run_cycle(p, MODE_CYCLE, base, target, U, W, last_token, draft, out, tau, p_draft,
-                   q_draft, nullptr, ws, stream);
+  return run_cycle(p, MODE_CYCLE, base, target, U, W, last_token, nullptr, draft, out, tau,
+                   p_draft, q_draft, nullptr, ws, stream);
+}
+
+spec_status spec_cycle_kb(const spec_params* p, const void* base, const void* target, const void* U,
+                          const void* W, const int32_t* last_token, const int32_t* verify_len,
+                          int32_t* draft, int32_t* out, int32_t* tau, float* p_draft,
+                          float* q_draft, void* ws, spec_stream_t stream) {
+  if (!verify_len) return SPEC_ERR_INVALID_ARG;
+  return run_cycle(p, MODE_CYCLE, base, target, U, W, last_token, verify_len, draft, out, tau,
+                   p_draft, q_draft, nullptr, ws, stream);
 }
 
 spec_status spec_verify_block(const spec_params* p, const void* target, const void* draft_logits,

@@ -74,6 +74,7 @@ struct ArgsTC {
   const __nv_bfloat16* U;
   const __nv_bfloat16* W;
   const int32_t* last_token;
+  const int32_t* vlen;   // [B] per-row verify length K_b (1..K), or null (K)
   int32_t* draft;
   int32_t* out;
   int32_t* tau;
@@ -124,6 +125,7 @@ struct CtlT {
   int32_t stoprow[N];
   int32_t tok[N];
   int32_t acc[N];        // accept outcome of the step, from the record tags
+  int32_t kb[N];         // verify length of each row of the group
   float zM[N], zS[N];    // draft statistics of the stop row
   float fMt[N], fSt[N];  // target statistics of the final row (stop row or row K)
   alignas(16) float4 fcst[N];  // final step: target max, 1 / target sum, draft max, 1 / draft sum
@@ -238,6 +240,11 @@ SPEC_DEV void bf16x8(const uint4& w, float* x) {
     x[2 * j] = __uint_as_float(u[j] << 16);
     x[2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
   }
+}
+
+// Verify length K_b of batch row b (K without a per-row array), clamped to 1..K.
+SPEC_DEV int row_verify_len(const int32_t* vlen, int64_t b, int K) {
+  return vlen ? min(max(__ldg(vlen + b), 1), K) : K;
 }
 
 template <typename T>
@@ -444,30 +451,30 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
           ok = false;
           break;
         }
-        const bool last = j == K - 1;
-        {  // the next job's target rows of this warp's rows into L2
-          const int nl2 = 2 * lane + tw;
-          if (j + 1 < K && nl2 < nb_g && nl2 < N &&
-              *reinterpret_cast<volatile int32_t*>(&ctl->alive[nl2]) != 0) {
-            const int64_t bb = (int64_t)g * N + nl2;
-            prefetch_l2_bulk(target + (bb * (K + 1) + j + 1) * V + vlo, bytes);
-            if (j + 2 == K) prefetch_l2_bulk(target + (bb * (K + 1) + K) * V + vlo, bytes);
-          }
-        }
-        // rows n = 2 l + tw still verifying (a snapshot: a row that stops
-        // meanwhile only costs an unused slice)
+        // this lane's row n = 2 l + tw and its verify length K_b
         const int nl = 2 * lane + tw;
-        const uint32_t rows = __ballot_sync(
-            FULL, nl < nb_g && nl < N &&
-                      (j == 0 || *reinterpret_cast<volatile int32_t*>(&ctl->alive[nl]) != 0));
-        // items: (row, target row j) and, at the last job, (row, target row K)
+        const bool inrow = nl < nb_g && nl < N;
+        const int kbl = inrow ? row_verify_len(a.vlen, (int64_t)g * N + nl, K) : 0;
+        const bool verifying =
+            inrow && j < kbl && (j == 0 || *reinterpret_cast<volatile int32_t*>(&ctl->alive[nl]) != 0);
+        if (verifying && j + 1 < kbl) {  // the next job's target rows of this row into L2
+          const int64_t bb = (int64_t)g * N + nl;
+          prefetch_l2_bulk(target + (bb * (K + 1) + j + 1) * V + vlo, bytes);
+          if (j + 2 == kbl) prefetch_l2_bulk(target + (bb * (K + 1) + kbl) * V + vlo, bytes);
+        }
+        // rows still verifying at position j (a snapshot: a row that stops
+        // meanwhile only costs an unused slice); items: (row, target row j)
+        // and, at a row's last verified position, (row, target row K_b)
+        const uint32_t rows = __ballot_sync(FULL, verifying);
+        const uint32_t lastm = __ballot_sync(FULL, verifying && j == kbl - 1);
         uint32_t imask = rows, cmask = rows;
         int isub = 0, csub = 0;
         auto next_item = [&](uint32_t& m, int& sub, int& n, int& trow) {
           if (!m) return false;
-          n = 2 * (__ffs(m) - 1) + tw;
-          trow = sub == 0 ? j : K;
-          if (last && sub == 0) {
+          const int l = __ffs(m) - 1;
+          n = 2 * l + tw;
+          trow = sub == 0 ? j : j + 1;
+          if (((lastm >> l) & 1u) && sub == 0) {
             sub = 1;
           } else {
             sub = 0;
@@ -699,13 +706,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
     // 3. warp 0 scans the bucket (kind 0: q_i, then the accept test against
     //    p_i; kind 2: the residual or the bonus row) and writes the outputs.
     auto draw_row = [&](int kind, int g, int par, int i, int n, int j) {
+      if (kind == 0 && i >= ctl->kb[n]) return;  // past the row's verify length: no draft
       RecT& rr = ctl->rrec[j];
       const int b = g * N + n;
       const int o = rr.owner;
       const float M = rr.M;
       const bool use_p = (rr.flags & 2) != 0;
       const bool alive = ctl->alive[n] != 0;
-      const int row = kind == 0 ? i : (alive ? K : ctl->stoprow[n]);
+      const int row = kind == 0 ? i : (alive ? ctl->kb[n] : ctl->stoprow[n]);
       if (warp == 0) {
         const int nbk_o = min(a.nc, a.nchunks - o * a.nc) * 4;
         const float tin = rr.trem;
@@ -832,14 +840,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
     constexpr int E = (kMaxG + 31) / 32;
     auto reduce_rows = [&](int kind, int g, int par, int i, int nb_g) {
       int mine = 0, local = 0;
-      const bool last = kind == 0 && i == K - 1;
       const int slot = kind == 0 ? i : K;  // partial and record slot
       for (int n = cta; n < nb_g; n += G, ++local) {
         ++mine;
         if ((local & 7) != warp) continue;  // warp-uniform
         const int b = g * N + n;
         const int c0 = lane * E;
-        const bool live = ctl->alive[n] != 0;
+        const int kbn = ctl->kb[n];
+        // verifying at this step; and this step is the row's last verified position
+        const bool live = ctl->alive[n] != 0 && (kind != 0 || i < kbn);
+        const bool last = kind == 0 && i == kbn - 1;
         RecT rc;
         rc.M = 0.f; rc.S = 1.f; rc.Mt = 0.f; rc.St = 1.f; rc.MtK = 0.f; rc.StK = 1.f;
         rc.trem = INFINITY; rc.owner = 0; rc.token = 0; rc.acc = 1; rc.flags = 0;
@@ -930,7 +940,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
             if (lane >= off) incl += y;
           }
           const float total = __shfl_sync(FULL, incl, 31);
-          const int row = kind == 0 ? i : (live ? K : ctl->stoprow[n]);
+          const int row = kind == 0 ? i : (live ? kbn : ctl->stoprow[n]);
           const float u = philox_uniform(a.seed, a.cycle, a.row0 + (uint32_t)b, (uint32_t)row,
                                          kind == 0 ? TAG_DRAFT : TAG_RESAMPLE);
           const float tgt = u * total;
@@ -961,16 +971,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         }
         if (kind == 0 && live) {
           target_row(i, rc.Mt, rc.St, rc.tam);
-          if (last) target_row(K, rc.MtK, rc.StK, rc.tamK);
+          if (last) target_row(kbn, rc.MtK, rc.StK, rc.tamK);  // the bonus row K_b
           if (a.greedy) {
             rc.acc = rc.tam == rc.token ? 1 : 0;
             if (lane == 0) {  // greedy step of a row still verifying
               a.out[(int64_t)b * (K + 1) + i] = rc.acc ? rc.token : rc.tam;
-              if (last && rc.acc) a.out[(int64_t)b * (K + 1) + K] = rc.tamK;
+              if (last && rc.acc) a.out[(int64_t)b * (K + 1) + kbn] = rc.tamK;
             }
           }
         }
-        if (kind == 0 && a.greedy && lane == 0 && a.draft) a.draft[(int64_t)b * K + i] = rc.token;
+        if (kind == 0 && a.greedy && lane == 0 && a.draft && i < kbn)
+          a.draft[(int64_t)b * K + i] = rc.token;
         if (lane == 0) ctl->rrec[local] = rc;
       }
       named_sync();
@@ -1031,12 +1042,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
       for (int n = tid; n < N; n += kComputeThreads) {
         ctl->alive[n] = n < nb_g ? 1 : 0;
         ctl->stoprow[n] = K;
+        int kbn = K;
+        if (n < nb_g && a.vlen) {
+          const int32_t raw = __ldg(a.vlen + g * N + n);
+          if (raw < 1 || raw > K) record_error(hdr, SPEC_ERR_INVALID_ARG, SITE_TOKEN_RANGE, g * N + n, raw);
+          kbn = min(max(raw, 1), K);
+        }
+        ctl->kb[n] = kbn;
       }
       if (cta == 0) {
         for (int idx = tid; idx < nb_g * K; idx += kComputeThreads) {
           const int64_t o = (int64_t)(g * N) * K + idx;
+          const int pos = idx % K;
+          const bool past = pos >= row_verify_len(a.vlen, (int64_t)g * N + idx / K, K);
           if (a.p_draft) a.p_draft[o] = NaNf;
-          if (a.q_draft && a.greedy) a.q_draft[o] = NaNf;
+          if (a.q_draft && (a.greedy || past)) a.q_draft[o] = NaNf;
+          if (a.draft && past) a.draft[o] = -1;
         }
       }
       // step 0's base and target logits of this CTA's slice into L2
@@ -1051,7 +1072,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
       mark(g, K + 1, 0);
 
       for (int i = 0; i < K; ++i) {
-        const bool last = i == K - 1;
         // ---------------- gather the Markov rows for this step
         mark(g, i, 0);
         for (int n = tid; n < N; n += kComputeThreads) {
@@ -1192,7 +1212,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         // accept outcomes from the tags; a row that stops (or the bonus at the
         // last step) reads its full record for the final step's statistics
         for (int n = tid; n < nb_g; n += kComputeThreads) {
-          if (ctl->alive[n] && (!ctl->acc[n] || last)) {
+          const bool lastn = i == ctl->kb[n] - 1;
+          if (ctl->alive[n] && i < ctl->kb[n] && (!ctl->acc[n] || lastn)) {
             const RecT r = load_rec(a.rec + ((int64_t)par * (K + 1) + i) * N + n);
             if (!ctl->acc[n]) {
               ctl->alive[n] = 0;
@@ -1202,7 +1223,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
               ctl->fMt[n] = r.Mt;  // target statistics of the stop row
               ctl->fSt[n] = r.St;
             } else {
-              ctl->fMt[n] = r.MtK;  // every draft accepted: the bonus comes from row K
+              ctl->fMt[n] = r.MtK;  // every draft accepted: the bonus comes from row K_b
               ctl->fSt[n] = r.StK;
             }
           }
@@ -1237,7 +1258,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         if (tid < nb_g) {  // the final rows of this CTA's slice into L2
           const int64_t b = (int64_t)g * N + tid;
           const bool alive = ctl->alive[tid] != 0;
-          const int row = alive ? K : ctl->stoprow[tid];
+          const int row = alive ? ctl->kb[tid] : ctl->stoprow[tid];
           prefetch_l2_bulk(target + (b * (K + 1) + row) * V + vslice_lo, slice_bytes);
           if (!alive) prefetch_l2_bulk(base + (b * K + row) * V + vslice_lo, slice_bytes);
         }
@@ -1245,7 +1266,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         {
           const bool rowok = nrow < nb_g;
           const bool ralive = rowok && ctl->alive[nrow] != 0;
-          const int frow = ralive ? K : (rowok ? ctl->stoprow[nrow] : 0);
+          const int frow = ralive ? ctl->kb[nrow] : (rowok ? ctl->stoprow[nrow] : 0);
           const int64_t brow = (int64_t)g * N + (rowok ? nrow : 0);
           const T* tsrc = target + (brow * (K + 1) + frow) * V;
           const T* bsrc = base + (brow * K + min(frow, K - 1)) * V;
@@ -1334,7 +1355,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
       if (cta == 0) {
         for (int n = tid; n < nb_g; n += kComputeThreads) {
           const int b = g * N + n;
-          const int j = ctl->alive[n] ? K : ctl->stoprow[n];
+          const int j = ctl->alive[n] ? ctl->kb[n] : ctl->stoprow[n];
           a.tau[b] = j + 1;
           for (int i2 = j + 1; i2 <= K; ++i2) a.out[(int64_t)b * (K + 1) + i2] = -1;
         }
@@ -1460,6 +1481,7 @@ cudaError_t launch_cycle_tc(const CycleLaunch& L, const CycleGeom& g, WsHeader* 
   a.U = reinterpret_cast<const __nv_bfloat16*>(L.U);
   a.W = reinterpret_cast<const __nv_bfloat16*>(L.W);
   a.last_token = L.last_token;
+  a.vlen = L.vlen;
   a.draft = L.draft;
   a.out = L.out;
   a.tau = L.tau;

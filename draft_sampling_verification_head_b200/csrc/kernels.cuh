@@ -64,6 +64,7 @@ struct CycleLaunch {
   const void* U;
   const void* W;
   const int32_t* last_token;
+  const int32_t* vlen;  // [B] per-row verify length K_b, or null (tensor-core cycle only)
   int32_t* draft;
   int32_t* out;
   int32_t* tau;

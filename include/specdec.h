@@ -145,6 +145,22 @@ spec_status spec_cycle(const spec_params *p, const void *base, const void *targe
                        int32_t *tau, float *p_draft, float *q_draft, void *workspace,
                        spec_stream_t stream);
 
+/* One cycle with a verify length per request (aigest.pl "DeepSeek prezentuje
+ * DSpark", section "Optymalizacja weryfikacji i wydajności": a scheduler fixes
+ * how many draft tokens of each request are verified, and its early stop keeps
+ * the method lossless).  verify_len [B] int32 (device): K_b in 1..K.  Row b
+ * drafts and verifies positions 0..K_b-1 and draws its bonus from target row
+ * K_b, so tau_b <= K_b + 1 and the draws are the full block's first K_b draws
+ * (the same random counters); draft[b, i] = -1 and q_draft[b, i] = NaN for
+ * i >= K_b, and target rows past K_b are never read.  A K_b outside 1..K is
+ * clamped and reported as SPEC_ERR_INVALID_ARG by spec_sync_status.  Tensor-core
+ * path only (bf16, rank a multiple of 64 up to 256); other shapes return
+ * SPEC_ERR_UNSUPPORTED.  spec_cycle is this call with every K_b = K. */
+spec_status spec_cycle_kb(const spec_params *p, const void *base, const void *target,
+                          const void *U, const void *W, const int32_t *last_token,
+                          const int32_t *verify_len, int32_t *draft, int32_t *out, int32_t *tau,
+                          float *p_draft, float *q_draft, void *workspace, spec_stream_t stream);
+
 /* spec_cycle without a workspace argument, for callers that cannot allocate
  * device memory when they run a cycle (code whose allocations all belong to a
  * framework pool, a host thread that must not call cudaMalloc because it

@@ -90,6 +90,23 @@ def make(w: Workload, B: int | None = None, seed: int | None = None):
     return dict(base=base, target=target, U=U, W=W, last_token=last)
 
 
+def make_loop(w: Workload, n_cycles: int, B: int | None = None, seed: int | None = None,
+              conf_range=(0.5, 1.0)):
+    """Inputs of a multi-cycle decode loop: base [C,B,K,V] and target
+    [C,B,K+1,V] (cycle c drawn as ``make`` with seed s + c), U, W and
+    last_token of cycle 0, and confidence scores conf [C,B,K] float32, uniform
+    over conf_range (a stand-in for a trained confidence head's outputs)."""
+    seed = w.seed if seed is None else seed
+    cyc = [make(w, B=B, seed=seed + 7919 * c) for c in range(n_cycles)]
+    B = cyc[0]["base"].shape[0]
+    g = torch.Generator().manual_seed(seed + 104729)
+    lo, hi = conf_range
+    conf = lo + (hi - lo) * torch.rand((n_cycles, B, w.K), generator=g, dtype=torch.float32)
+    return dict(base=torch.stack([d["base"] for d in cyc]),
+                target=torch.stack([d["target"] for d in cyc]),
+                U=cyc[0]["U"], W=cyc[0]["W"], last_token=cyc[0]["last_token"], conf=conf)
+
+
 def to_numpy_raw(t: torch.Tensor) -> np.ndarray:
     """Raw storage for the oracle: bf16 as uint16 bit patterns, f32 as float32."""
     t = t.contiguous()

@@ -30,6 +30,8 @@ _SIGS = {
     "spec_verify_block": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_cycle": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_cycle_kb": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "spec_decode_loop": (ctypes.c_int, [_P, ctypes.c_int32, _P, _P, _P, ctypes.c_float, _P, _P, _P,
+                                         _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_sync_status": (ctypes.c_int, [_P, _P]),
     "spec_cycle_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_l2_persist": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
@@ -175,6 +177,19 @@ def cycle_kb(p: Params, base, target, U, W, last_token, verify_len, draft, out, 
                                _stream(stream)), "spec_cycle_kb")
 
 
+def decode_loop(p: Params, n_cycles, base, target, U, W, last_token, draft, out, tau, p_draft,
+                q_draft, next_token, ws, conf=None, conf_threshold=0.0, verify_len=None,
+                stream=None):
+    """spec_decode_loop: n_cycles chained cycles in one launch; inputs and
+    outputs carry a leading cycle axis, next_token [B] the last cycle's last
+    emitted tokens."""
+    _check(lib().spec_decode_loop(ctypes.byref(p.c()), int(n_cycles), _ptr(base), _ptr(target),
+                                  _ptr(conf), float(conf_threshold), _ptr(verify_len), _ptr(U),
+                                  _ptr(W), _ptr(last_token), _ptr(draft), _ptr(out), _ptr(tau),
+                                  _ptr(p_draft), _ptr(q_draft), _ptr(next_token), _ptr(ws),
+                                  _stream(stream)), "spec_decode_loop")
+
+
 def cycle_noalloc(p: Params, base, target, U, W, last_token, draft, out, tau, p_draft, q_draft,
                   status_out=None, stream=None):
     """spec_cycle on the library's built-in scratch array (no workspace)."""
@@ -210,11 +225,12 @@ def debug_curand_philox(ctr, key, out, stream=None):
                                           _stream(stream)), "spec_debug_curand_philox")
 
 
-def alloc_outputs(p: Params, device="cuda"):
-    """Output tensors for one cycle."""
+def alloc_outputs(p: Params, device="cuda", n_cycles=None):
+    """Output tensors for one cycle, or with a leading axis of n_cycles."""
     import torch
-    return dict(draft=torch.full((p.B, p.K), -7, dtype=torch.int32, device=device),
-                out=torch.full((p.B, p.K + 1), -7, dtype=torch.int32, device=device),
-                tau=torch.zeros(p.B, dtype=torch.int32, device=device),
-                p_draft=torch.full((p.B, p.K), -1.0, dtype=torch.float32, device=device),
-                q_draft=torch.full((p.B, p.K), -1.0, dtype=torch.float32, device=device))
+    lead = () if n_cycles is None else (int(n_cycles),)
+    return dict(draft=torch.full(lead + (p.B, p.K), -7, dtype=torch.int32, device=device),
+                out=torch.full(lead + (p.B, p.K + 1), -7, dtype=torch.int32, device=device),
+                tau=torch.zeros(lead + (p.B,), dtype=torch.int32, device=device),
+                p_draft=torch.full(lead + (p.B, p.K), -1.0, dtype=torch.float32, device=device),
+                q_draft=torch.full(lead + (p.B, p.K), -1.0, dtype=torch.float32, device=device))

@@ -2,6 +2,7 @@
 // workspace layout, tensor maps and launches.  No allocation happens here.
 #include <curand_kernel.h>
 
+#include <climits>
 #include <cstdio>
 #include <cstring>
 
@@ -16,6 +17,7 @@ namespace {
 thread_local int32_t g_last_launches = 0;
 
 constexpr uint64_t kDefaultSpin = 4000000ull;  // polls of ~0.5 us back-off: about 2 s
+constexpr int32_t kMaxLoopCycles = 1 << 16;     // record tags of one launch stay below 2^31
 
 int num_sms() {
   int dev = 0, n = 0;
@@ -219,11 +221,21 @@ spec_status spec_markov_bias(const spec_params* p, const void* U, const void* W,
 }
 
 // The fused cycle on the tensor-core path (geometry already decided).
+// Loop inputs of the tensor-core cycle: cycles per launch, confidence scores
+// with their threshold, and the carried last tokens (one cycle: all unset).
+struct LoopInputs {
+  int ncyc = 1;
+  const float* conf = nullptr;
+  float conf_thr = 0.f;
+  int32_t* next_token = nullptr;
+};
+
 static spec_status run_cycle_tc(const spec_params* p, const CycleGeom& g, const void* base,
                                 const void* target, const void* U, const void* W,
                                 const int32_t* last_token, const int32_t* vlen, int32_t* draft,
                                 int32_t* out, int32_t* tau, float* p_draft, float* q_draft,
-                                void* ws, spec_stream_t stream) {
+                                void* ws, spec_stream_t stream,
+                                const LoopInputs& loop = LoopInputs()) {
   CUtensorMap tmW;
   if (!make_tmap_W(&tmW, W, p->r, p->V, kCycleWBoxK)) return SPEC_ERR_CUDA;
   CycleLaunch L;
@@ -234,6 +246,10 @@ static spec_status run_cycle_tc(const spec_params* p, const CycleGeom& g, const 
   L.W = W;
   L.last_token = last_token;
   L.vlen = vlen;
+  L.conf = loop.conf;
+  L.conf_thr = loop.conf_thr;
+  L.next_token = loop.next_token;
+  L.ncyc = loop.ncyc;
   L.draft = draft;
   L.out = out;
   L.tau = tau;
@@ -355,6 +371,41 @@ spec_status spec_cycle_kb(const spec_params* p, const void* base, const void* ta
   if (!verify_len) return SPEC_ERR_INVALID_ARG;
   return run_cycle(p, MODE_CYCLE, base, target, U, W, last_token, verify_len, draft, out, tau,
                    p_draft, q_draft, nullptr, ws, stream);
+}
+
+spec_status spec_decode_loop(const spec_params* p, int32_t n_cycles, const void* base,
+                             const void* target, const float* conf, float conf_threshold,
+                             const int32_t* verify_len, const void* U, const void* W,
+                             const int32_t* last_token, int32_t* draft, int32_t* out, int32_t* tau,
+                             float* p_draft, float* q_draft, int32_t* next_token, void* ws,
+                             spec_stream_t stream) {
+  g_last_launches = 0;
+  spec_status s = check_params(p);
+  if (s != SPEC_OK) return s;
+  if (n_cycles < 1 || n_cycles > kMaxLoopCycles || (conf && verify_len)) return SPEC_ERR_INVALID_ARG;
+  if (n_cycles > 1 && !next_token) return SPEC_ERR_INVALID_ARG;
+  if ((int64_t)n_cycles * p->B > INT32_MAX) return SPEC_ERR_INVALID_ARG;
+  if (!base || !target || !last_token || !out || !tau || !U || !W || p->r < 1)
+    return SPEC_ERR_INVALID_ARG;
+  if (!aligned16(base) || !aligned16(target) || !aligned16(U) || !aligned16(W))
+    return SPEC_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SPEC_ERR_WORKSPACE;
+  const int sms = num_sms();
+  if (sms <= 0) return SPEC_ERR_CUDA;
+  CycleGeom g;
+  const char* why = nullptr;
+  if (!cycle_tc_geometry(p->B, p->K, p->V, p->r, p->dtype, p->flags, sms, &g, &why)) {
+    fprintf(stderr, "specdec: the decode loop needs the tensor-core cycle (bf16, rank a multiple "
+                    "of 64 up to 256): %s\n", why);
+    return SPEC_ERR_UNSUPPORTED;
+  }
+  LoopInputs loop;
+  loop.ncyc = n_cycles;
+  loop.conf = conf;
+  loop.conf_thr = conf_threshold;
+  loop.next_token = next_token;
+  return run_cycle_tc(p, g, base, target, U, W, last_token, verify_len, draft, out, tau, p_draft,
+                      q_draft, ws, stream, loop);
 }
 
 spec_status spec_verify_block(const spec_params* p, const void* target, const void* draft_logits,

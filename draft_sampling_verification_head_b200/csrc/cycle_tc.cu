@@ -74,7 +74,9 @@ struct ArgsTC {
   const __nv_bfloat16* U;
   const __nv_bfloat16* W;
   const int32_t* last_token;
-  const int32_t* vlen;   // [B] per-row verify length K_b (1..K), or null (K)
+  const int32_t* vlen;   // [C][B] per-row verify length K_b (1..K), or null
+  const float* conf;     // [C][B][K] confidence scores (used without vlen), or null
+  int32_t* next_token;   // [B] each row's last emitted token (carried between cycles), or null
   int32_t* draft;
   int32_t* out;
   int32_t* tau;
@@ -90,6 +92,8 @@ struct ArgsTC {
   uint64_t* trace;   // [K+2][kTracePhases] device timeline of CTA 0, or null
   int B, K, V, r, G, nc, nchunks, greedy, ngroups, NT;
   float k;           // log2(e) / T (1 in greedy mode)
+  float conf_thr;    // prefix survival a verified position needs (with conf)
+  int ncyc;          // cycles C run by this launch, one after another
   uint64_t seed, cycle, spin;
   uint32_t row0;     // global index of batch row 0 (Philox counter word 1)
   int nbk;           // buckets per CTA (4 per chunk)
@@ -242,9 +246,23 @@ SPEC_DEV void bf16x8(const uint4& w, float* x) {
   }
 }
 
-// Verify length K_b of batch row b (K without a per-row array), clamped to 1..K.
-SPEC_DEV int row_verify_len(const int32_t* vlen, int64_t b, int K) {
-  return vlen ? min(max(__ldg(vlen + b), 1), K) : K;
+// Verify length K_b of row gb (cycle-major row index c * B + b): the given
+// length clamped to 1..K; or, from confidence scores, the number of leading
+// positions whose prefix survival (fp32 product of the scores of positions
+// 0..i, in position order) is at least the threshold, at least 1; else K.
+SPEC_DEV int row_verify_len(const ArgsTC& a, int64_t gb) {
+  const int K = a.K;
+  if (a.vlen) return min(max(__ldg(a.vlen + gb), 1), K);
+  if (!a.conf) return K;
+  const float* c = a.conf + gb * K;
+  float s = 1.f;
+  int kb = 0;
+  for (int i = 0; i < K; ++i) {
+    s = __fmul_rn(s, __ldg(c + i));
+    if (!(s >= a.conf_thr)) break;  // a NaN score ends the prefix too
+    kb = i + 1;
+  }
+  return max(kb, 1);
 }
 
 template <typename T>
@@ -281,6 +299,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
   const int ntc = min(a.NT, ncc);                 // of which in tensor memory
   const int has_final = a.greedy ? 0 : 1;
   const int nrounds = K + has_final;              // MMA rounds per group
+  // jobs: (cycle, group) pairs in cycle-major order; rows of job t are
+  // c * B + g * N + n in the inputs and outputs (c = t / ngroups, g = t % ngroups)
+  const int njobs = a.ngroups * a.ncyc;
   WsHeader* hdr = a.hdr;
   const T* base = a.base;
   const T* target = a.target;
@@ -350,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
       };
       for (int c = 0; c < ntc && ok; ++c)
         for (int s = 0; s < nkb && ok; ++s) load_stage(c, s, pol_once);
-      for (int g = 0; g < a.ngroups && ok; ++g)
+      for (int t = 0; t < njobs && ok; ++t)
         for (int rd = 0; rd < nrounds && ok; ++rd)
           for (int c = ntc; c < ncc && ok; ++c)
             for (int s = 0; s < nkb && ok; ++s) load_stage(c, s, pol_stream);
@@ -370,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
       bool ok = mbar_wait_bounded(&ctl->tready, 0, a.spin, &hdr->abort);
       if (!ok) record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_BREADY, cta, -1);
       tc_fence_after();
-      for (int g = 0; g < a.ngroups && ok; ++g) {
+      for (int t = 0; t < njobs && ok; ++t) {
         for (int rd = 0; rd < nrounds && ok; ++rd, ++rd_ctr) {
           if (!mbar_wait_bounded(&ctl->bready, rd_ctr & 1, a.spin, &hdr->abort)) {
             record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_BREADY, cta, rd);
@@ -378,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
             break;
           }
           tc_fence_after();
-          if (a.trace && cta == 0 && g == 0) a.trace[(size_t)min(rd, K) * kTracePhases + 9] = globaltimer_ns();
+          if (a.trace && cta == 0 && t == 0) a.trace[(size_t)min(rd, K) * kTracePhases + 9] = globaltimer_ns();
           for (int c = 0; c < ncc && ok; ++c, ++cc) {
             const uint32_t b = cc & 1;
             if (cc >= 2 &&
@@ -420,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
             }
             umma_commit(&ctl->dfull[b]);
           }
-          if (a.trace && cta == 0 && g == 0) a.trace[(size_t)min(rd, K) * kTracePhases + 10] = globaltimer_ns();
+          if (a.trace && cta == 0 && t == 0) a.trace[(size_t)min(rd, K) * kTracePhases + 10] = globaltimer_ns();
         }
       }
       umma_commit(&ctl->mmadone);
@@ -442,8 +463,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
     const uint64_t pol = policy_evict_first();
     uint32_t tu = 0, tcn = 0, J = 0;  // copies issued, copies consumed, jobs
     bool ok = true;
-    for (int g = 0; g < a.ngroups && ok; ++g) {
-      const int par = g & 1;
+    for (int t = 0; t < njobs && ok; ++t) {
+      const int g = t % a.ngroups, par = t & 1;
+      const int64_t gb0 = (int64_t)(t / a.ngroups) * a.B + (int64_t)g * N;  // row 0 of the job
       const int nb_g = min(N, a.B - g * N);
       for (int j = 0; j < K && ok; ++j, ++J) {
         if (!mbar_wait_bounded(&ctl->tgo, J & 1, a.spin, &hdr->abort)) {
@@ -454,11 +476,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         // this lane's row n = 2 l + tw and its verify length K_b
         const int nl = 2 * lane + tw;
         const bool inrow = nl < nb_g && nl < N;
-        const int kbl = inrow ? row_verify_len(a.vlen, (int64_t)g * N + nl, K) : 0;
+        const int kbl = inrow ? row_verify_len(a, gb0 + nl) : 0;
         const bool verifying =
             inrow && j < kbl && (j == 0 || *reinterpret_cast<volatile int32_t*>(&ctl->alive[nl]) != 0);
         if (verifying && j + 1 < kbl) {  // the next job's target rows of this row into L2
-          const int64_t bb = (int64_t)g * N + nl;
+          const int64_t bb = gb0 + nl;
           prefetch_l2_bulk(target + (bb * (K + 1) + j + 1) * V + vlo, bytes);
           if (j + 2 == kbl) prefetch_l2_bulk(target + (bb * (K + 1) + kbl) * V + vlo, bytes);
         }
@@ -489,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
           if (lane == 0) {
             mbar_arrive_expect_tx(&ctl->tfull[tw][slot], bytes);
             bulk_load(ring + slot * rslot,
-                      target + (((int64_t)g * N + n) * (K + 1) + trow) * V + vlo, bytes,
+                      target + ((gb0 + n) * (K + 1) + trow) * V + vlo, bytes,
                       &ctl->tfull[tw][slot], pol);
           }
           ++tu;
@@ -570,6 +592,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
     uint32_t cc = 0, nbar = 0;
     const uint32_t ev0 = ld_volatile_u32(&hdr->events);  // record tags of this launch start here
     bool failed = false;
+    // the current job: index, cycle of the launch, first row (cycle-major), Philox cycle
+    int jt = 0, jcy = 0;
+    int64_t jb0 = 0;
+    uint64_t jcyc = a.cycle;
+    // the committed token row b's block starts from: the given last token in
+    // the first cycle, then the last token the row emitted in the cycle before
+    auto first_token = [&](int b) -> int32_t {
+      return jcy == 0 ? __ldg(a.last_token + b) : __ldcg(a.next_token + b);
+    };
+    // the row's last emitted token of this cycle: carried to the next cycle
+    auto emit_last = [&](int b, int32_t tok) {
+      if (a.next_token) a.next_token[b] = tok;
+    };
     auto soft_fail = [&](int code, int site, int x, int y) {
       record_error(hdr, code, site, x, y);
       ctl->abort_local = 1;
@@ -596,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
     const uint32_t slice_bytes = (uint32_t)((vslice_hi - vslice_lo) * sizeof(T));
     uint64_t* trace = (a.trace != nullptr && cta == 0 && tid == 0) ? a.trace : nullptr;
     auto mark = [&](int g, int step, int phase) {
-      if (trace && g == 0) trace[(size_t)step * kTracePhases + phase] = globaltimer_ns();
+      if (trace && g == 0 && jt == 0) trace[(size_t)step * kTracePhases + phase] = globaltimer_ns();
     };
 
     // ---- W^T of the resident chunks into tensor memory (once per launch).
@@ -709,6 +744,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
       if (kind == 0 && i >= ctl->kb[n]) return;  // past the row's verify length: no draft
       RecT& rr = ctl->rrec[j];
       const int b = g * N + n;
+      const int64_t gb = jb0 + n;
       const int o = rr.owner;
       const float M = rr.M;
       const bool use_p = (rr.flags & 2) != 0;
@@ -760,11 +796,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
       float tv = 0.f, bv = 0.f;
       if (warp == 0) {  // the row's logits at the bucket's tokens, in flight meanwhile
         if (kind == 0) {
-          bv = ld_elem(base, ((int64_t)b * K + i) * V + vc);
-          tv = ld_elem(target, ((int64_t)b * (K + 1) + i) * V + vc);
+          bv = ld_elem(base, (gb * K + i) * V + vc);
+          tv = ld_elem(target, (gb * (K + 1) + i) * V + vc);
         } else {
-          tv = ld_elem(target, ((int64_t)b * (K + 1) + row) * V + vc);
-          if (!alive) bv = ld_elem(base, ((int64_t)b * K + row) * V + vc);
+          tv = ld_elem(target, (gb * (K + 1) + row) * V + vc);
+          if (!alive) bv = ld_elem(base, (gb * K + row) * V + vc);
         }
       }
       {  // warp w: rank rows [w*ks, w*ks + ks)
@@ -799,7 +835,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
             pd = fexp2((td - rr.Mt) * k) / rr.St;
             const float ratio = fexp2(((td - rr.Mt) - (zd - M)) * k) * (S / rr.St);
             const float uacc =
-                philox_uniform(a.seed, a.cycle, a.row0 + (uint32_t)b, (uint32_t)i, TAG_ACCEPT);
+                philox_uniform(a.seed, jcyc, a.row0 + (uint32_t)b, (uint32_t)i, TAG_ACCEPT);
             accept = uacc < fminf(ratio, 1.0f) ? 1 : 0;
           }
           if (lane == 0) {
@@ -807,11 +843,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
             rr.token = d;
             rr.acc = accept;
             a.tokens[((int64_t)par * K + i) * N + n] = d;
-            if (a.draft) a.draft[(int64_t)b * K + i] = d;
-            if (a.q_draft) a.q_draft[(int64_t)b * K + i] = qd;
+            if (a.draft) a.draft[gb * K + i] = d;
+            if (a.q_draft) a.q_draft[gb * K + i] = qd;
             if (alive) {
-              if (a.p_draft) a.p_draft[(int64_t)b * K + i] = pd;
-              if (accept) a.out[(int64_t)b * (K + 1) + i] = d;
+              if (a.p_draft) a.p_draft[gb * K + i] = pd;
+              if (accept) a.out[gb * (K + 1) + i] = d;
             }
           }
         } else {  // the same expressions as the final epilogue's bucket masses
@@ -822,7 +858,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
           const int wl = bucket_scan(w, ctl->dtin);
           if (lane == 0) {
             rr.token = v0 + wl;
-            a.out[(int64_t)b * (K + 1) + row] = v0 + wl;
+            a.out[gb * (K + 1) + row] = v0 + wl;
+            emit_last(b, v0 + wl);
           }
         }
       }
@@ -845,6 +882,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         ++mine;
         if ((local & 7) != warp) continue;  // warp-uniform
         const int b = g * N + n;
+        const int64_t gb = jb0 + n;
         const int c0 = lane * E;
         const int kbn = ctl->kb[n];
         // verifying at this step; and this step is the row's last verified position
@@ -941,7 +979,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
           }
           const float total = __shfl_sync(FULL, incl, 31);
           const int row = kind == 0 ? i : (live ? kbn : ctl->stoprow[n]);
-          const float u = philox_uniform(a.seed, a.cycle, a.row0 + (uint32_t)b, (uint32_t)row,
+          const float u = philox_uniform(a.seed, jcyc, a.row0 + (uint32_t)b, (uint32_t)row,
                                          kind == 0 ? TAG_DRAFT : TAG_RESAMPLE);
           const float tgt = u * total;
           float cum = incl - loc, before = 0.f;
@@ -975,13 +1013,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
           if (a.greedy) {
             rc.acc = rc.tam == rc.token ? 1 : 0;
             if (lane == 0) {  // greedy step of a row still verifying
-              a.out[(int64_t)b * (K + 1) + i] = rc.acc ? rc.token : rc.tam;
-              if (last && rc.acc) a.out[(int64_t)b * (K + 1) + kbn] = rc.tamK;
+              a.out[gb * (K + 1) + i] = rc.acc ? rc.token : rc.tam;
+              if (last && rc.acc) a.out[gb * (K + 1) + kbn] = rc.tamK;
+              if (!rc.acc) emit_last(b, rc.tam);
+              else if (last) emit_last(b, rc.tamK);
             }
           }
         }
         if (kind == 0 && a.greedy && lane == 0 && a.draft && i < kbn)
-          a.draft[(int64_t)b * K + i] = rc.token;
+          a.draft[gb * K + i] = rc.token;
         if (lane == 0) ctl->rrec[local] = rc;
       }
       named_sync();
@@ -994,7 +1034,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         const RecT& rc = ctl->rrec[tid];
         const size_t at = ((size_t)par * (K + 1) + slot) * N + n;
         store_rec(a.rec + at, rc);
-        const uint32_t tag = ev0 + (uint32_t)(g * (K + 1) + slot + 1);
+        const uint32_t tag = ev0 + (uint32_t)(jt * (K + 1) + slot + 1);
         st_release_u64(a.rtag + at, ((uint64_t)tag << 32) | ((uint64_t)(rc.acc & 1) << 31) |
                                         (uint64_t)(uint32_t)(rc.token & 0x7fffffff));
       }
@@ -1002,10 +1042,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
     };
     // Wait until every row's record of this slot carries this step's tag;
     // thread n < nb_g polls row n.  Returns false if the launch is aborted.
-    auto records_hop = [&](int g, int par, int slot, int nb_g) {
+    auto records_hop = [&](int job, int par, int slot, int nb_g) {
       if (tid < nb_g) {
         const uint64_t* t = a.rtag + ((size_t)par * (K + 1) + slot) * N + tid;
-        const uint32_t want = ev0 + (uint32_t)(g * (K + 1) + slot + 1);
+        const uint32_t want = ev0 + (uint32_t)(job * (K + 1) + slot + 1);
         bool ok = false;
         for (uint64_t it = 0; it < a.spin; ++it) {
           const uint64_t wv = ld_acquire_u64(t);
@@ -1036,25 +1076,31 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
       }
     };
 
-    for (int g = 0; g < a.ngroups && !failed; ++g) {
-      const int par = g & 1;
+    for (int t = 0; t < njobs && !failed; ++t) {
+      const int g = t % a.ngroups, par = t & 1;
       const int nb_g = min(N, a.B - g * N);
+      jt = t;
+      jcy = t / a.ngroups;
+      jb0 = (int64_t)jcy * a.B + (int64_t)g * N;
+      jcyc = a.cycle + (uint64_t)jcy;
       for (int n = tid; n < N; n += kComputeThreads) {
         ctl->alive[n] = n < nb_g ? 1 : 0;
         ctl->stoprow[n] = K;
         int kbn = K;
-        if (n < nb_g && a.vlen) {
-          const int32_t raw = __ldg(a.vlen + g * N + n);
-          if (raw < 1 || raw > K) record_error(hdr, SPEC_ERR_INVALID_ARG, SITE_TOKEN_RANGE, g * N + n, raw);
-          kbn = min(max(raw, 1), K);
+        if (n < nb_g) {
+          if (a.vlen) {
+            const int32_t raw = __ldg(a.vlen + jb0 + n);
+            if (raw < 1 || raw > K) record_error(hdr, SPEC_ERR_INVALID_ARG, SITE_TOKEN_RANGE, g * N + n, raw);
+          }
+          kbn = row_verify_len(a, jb0 + n);
         }
         ctl->kb[n] = kbn;
       }
       if (cta == 0) {
         for (int idx = tid; idx < nb_g * K; idx += kComputeThreads) {
-          const int64_t o = (int64_t)(g * N) * K + idx;
+          const int64_t o = jb0 * K + idx;
           const int pos = idx % K;
-          const bool past = pos >= row_verify_len(a.vlen, (int64_t)g * N + idx / K, K);
+          const bool past = pos >= row_verify_len(a, jb0 + idx / K);
           if (a.p_draft) a.p_draft[o] = NaNf;
           if (a.q_draft && (a.greedy || past)) a.q_draft[o] = NaNf;
           if (a.draft && past) a.draft[o] = -1;
@@ -1062,13 +1108,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
       }
       // step 0's base and target logits of this CTA's slice into L2
       if (tid < nb_g) {
-        const int64_t b = (int64_t)g * N + tid;
+        const int64_t b = jb0 + tid;
         prefetch_l2_bulk(base + b * K * V + vslice_lo, slice_bytes);
         prefetch_l2_bulk(target + b * (K + 1) * V + vslice_lo, slice_bytes);
         if (K == 1) prefetch_l2_bulk(target + (b * (K + 1) + 1) * V + vslice_lo, slice_bytes);
       }
       named_sync();
-      if (tid == 0 && g > 0) mbar_arrive(&ctl->tgo);  // the target warps may take row 0 of this group
+      if (tid == 0 && t > 0) mbar_arrive(&ctl->tgo);  // the target warps may take row 0 of this group
       mark(g, K + 1, 0);
 
       for (int i = 0; i < K; ++i) {
@@ -1077,7 +1123,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         for (int n = tid; n < N; n += kComputeThreads) {
           int p = 0;
           if (n < nb_g) {
-            p = (i == 0) ? __ldg(a.last_token + g * N + n) : ctl->tok[n];
+            p = (i == 0) ? first_token(g * N + n) : ctl->tok[n];
             if (p < 0 || p >= V) {
               record_error(hdr, SPEC_ERR_TOKEN_RANGE, SITE_TOKEN_RANGE, g * N + n, p);
               p = 0;
@@ -1089,13 +1135,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         gather_u(nb_g);
         // the next step's base logits into L2 while this step runs
         if (tid < nb_g && i + 1 < K)
-          prefetch_l2_bulk(base + (((int64_t)g * N + tid) * K + i + 1) * V + vslice_lo, slice_bytes);
+          prefetch_l2_bulk(base + ((jb0 + tid) * K + i + 1) * V + vslice_lo, slice_bytes);
         mark(g, i, 1);
 
         // ---------------- epilogue: z = bias + base, exact bucket statistics
         {
           const bool rowok = nrow < nb_g;
-          const int64_t brow = (int64_t)g * N + (rowok ? nrow : 0);
+          const int64_t brow = jb0 + (rowok ? nrow : 0);
           const T* bsrc = base + (brow * K + i) * V;
           float pm = -INFINITY, ps = 0.f;  // stochastic: (max, sum); greedy: arg-max value
           int32_t pi = 0x7fffffff;         // greedy: arg-max index
@@ -1205,7 +1251,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         if (a.trace && g == 0 && tid == 0 && mine)
           atomicMax(reinterpret_cast<unsigned long long*>(a.trace) + (size_t)i * kTracePhases + 7,
                     (unsigned long long)globaltimer_ns());
-        if (!records_hop(g, par, i, nb_g)) {
+        if (!records_hop(t, par, i, nb_g)) {
           failed = true;
           break;
         }
@@ -1244,7 +1290,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
           int p = 0;
           if (n < nb_g && !ctl->alive[n]) {
             const int j = ctl->stoprow[n];
-            p = j == 0 ? __ldg(a.last_token + g * N + n)
+            p = j == 0 ? first_token(g * N + n)
                        : __ldcg(a.tokens + ((int64_t)par * K + (j - 1)) * N + n);
             if (p < 0 || p >= V) p = 0;
           }
@@ -1256,7 +1302,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         named_sync();
         gather_u(nb_g);
         if (tid < nb_g) {  // the final rows of this CTA's slice into L2
-          const int64_t b = (int64_t)g * N + tid;
+          const int64_t b = jb0 + tid;
           const bool alive = ctl->alive[tid] != 0;
           const int row = alive ? ctl->kb[tid] : ctl->stoprow[tid];
           prefetch_l2_bulk(target + (b * (K + 1) + row) * V + vslice_lo, slice_bytes);
@@ -1267,7 +1313,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
           const bool rowok = nrow < nb_g;
           const bool ralive = rowok && ctl->alive[nrow] != 0;
           const int frow = ralive ? ctl->kb[nrow] : (rowok ? ctl->stoprow[nrow] : 0);
-          const int64_t brow = (int64_t)g * N + (rowok ? nrow : 0);
+          const int64_t brow = jb0 + (rowok ? nrow : 0);
           const T* tsrc = target + (brow * (K + 1) + frow) * V;
           const T* bsrc = base + (brow * K + min(frow, K - 1)) * V;
           const float4 c = rowok ? ctl->fcst[nrow] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1344,8 +1390,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         mark(g, K, 4);
         // the reducers draw each row's residual / bonus token and write it
         reduce_rows(2, g, par, K, nb_g);
-        // the next group overwrites the bucket statistics: every draw is done first
-        if (g + 1 < a.ngroups && !records_hop(g, par, K, nb_g)) {
+        // the next job overwrites the bucket statistics, and the next cycle
+        // starts from the tokens drawn here: every draw is done first
+        if (t + 1 < njobs && !records_hop(t, par, K, nb_g)) {
           failed = true;
           break;
         }
@@ -1354,16 +1401,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
       // tau and the -1 padding after it
       if (cta == 0) {
         for (int n = tid; n < nb_g; n += kComputeThreads) {
-          const int b = g * N + n;
+          const int64_t b = jb0 + n;
           const int j = ctl->alive[n] ? ctl->kb[n] : ctl->stoprow[n];
           a.tau[b] = j + 1;
-          for (int i2 = j + 1; i2 <= K; ++i2) a.out[(int64_t)b * (K + 1) + i2] = -1;
+          for (int i2 = j + 1; i2 <= K; ++i2) a.out[b * (K + 1) + i2] = -1;
         }
       }
       named_sync();
       mark(g, K, 6);
       if (ctl->abort_local) failed = true;
-    }  // groups
+    }  // jobs
     (void)soft_fail;
   }
 
@@ -1385,7 +1432,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
       hdr->bar = 0;
       hdr->rec = 0;
       hdr->abort = 0;
-      hdr->events += (uint32_t)(a.ngroups * (K + 1));  // tags of the next launch differ
+      hdr->events += (uint32_t)(njobs * (K + 1));  // tags of the next launch differ
       __threadfence();
       atomicExch(&hdr->exit_count, 0u);
     }
@@ -1482,6 +1529,8 @@ cudaError_t launch_cycle_tc(const CycleLaunch& L, const CycleGeom& g, WsHeader* 
   a.W = reinterpret_cast<const __nv_bfloat16*>(L.W);
   a.last_token = L.last_token;
   a.vlen = L.vlen;
+  a.conf = L.conf;
+  a.next_token = L.next_token;
   a.draft = L.draft;
   a.out = L.out;
   a.tau = L.tau;
@@ -1515,6 +1564,8 @@ cudaError_t launch_cycle_tc(const CycleLaunch& L, const CycleGeom& g, WsHeader* 
   a.ngroups = (L.B + g.N - 1) / g.N;
   a.NT = std::min(kMaxNT, g.nc);
   a.k = L.greedy ? 1.0f : 1.4426950408889634f / L.temperature;
+  a.conf_thr = L.conf_thr;
+  a.ncyc = std::max(L.ncyc, 1);
   a.seed = L.seed;
   a.row0 = L.row0;
   a.cycle = L.cycle;

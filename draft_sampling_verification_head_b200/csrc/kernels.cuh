@@ -64,7 +64,11 @@ struct CycleLaunch {
   const void* U;
   const void* W;
   const int32_t* last_token;
-  const int32_t* vlen;  // [B] per-row verify length K_b, or null (tensor-core cycle only)
+  const int32_t* vlen;  // [C][B] per-row verify length K_b, or null (tensor-core cycle only)
+  const float* conf;    // [C][B][K] confidence scores, or null (tensor-core cycle only)
+  float conf_thr;       // prefix survival threshold for conf
+  int32_t* next_token;  // [B] last emitted token per row, carried between cycles, or null
+  int ncyc;             // cycles per launch (0 or 1: one)
   int32_t* draft;
   int32_t* out;
   int32_t* tau;

@@ -161,6 +161,39 @@ spec_status spec_cycle_kb(const spec_params *p, const void *base, const void *ta
                           const int32_t *verify_len, int32_t *draft, int32_t *out, int32_t *tau,
                           float *p_draft, float *q_draft, void *workspace, spec_stream_t stream);
 
+/* A decode loop: n_cycles cycles in one persistent launch (aigest.pl "DeepSeek
+ * prezentuje DSpark", section "Jak działa spekulatywne dekodowanie DSpark?":
+ * decoding repeats draft-and-verify cycles, each costing T_draft + T_verify
+ * for its tau tokens).  The token a row emits last in cycle c (its correction
+ * or its bonus token) is the committed token cycle c + 1 starts from, and
+ * cycle c draws with Philox cycle counter p->cycle + c; cycle c is otherwise
+ * spec_cycle_kb on slice c of the inputs.  Its verify lengths come from
+ * verify_len, or from confidence scores (section "Optymalizacja weryfikacji i
+ * wydajności": a score per draft position estimating the chance that its
+ * token survives verification given accepted predecessors): K_b is the number
+ * of leading positions whose prefix survival, the fp32 product of the scores
+ * of positions 0..i taken in position order, is >= conf_threshold, and at
+ * least 1 (a NaN score ends the prefix); or K with neither.
+ *   base        [C, B, K, V]    dtype   (C = n_cycles; slice c feeds cycle c)
+ *   target      [C, B, K+1, V]  dtype
+ *   conf        [C, B, K]       float   or NULL
+ *   verify_len  [C, B]          int32   or NULL (not both with conf)
+ *   U, W, last_token            as for spec_cycle (last_token: cycle 0's)
+ *   draft, p_draft, q_draft [C, B, K]; out [C, B, K+1]; tau [C, B]
+ *   next_token  [B]             int32   the last token each row emitted in the
+ *               last cycle (the next call's last_token); required when
+ *               n_cycles > 1 (it carries the tokens between cycles), and it
+ *               may be the same buffer as last_token.
+ * n_cycles is 1..65536.  Tensor-core path only (bf16, rank a multiple of 64 up
+ * to 256); other shapes return SPEC_ERR_UNSUPPORTED.  Device-side errors are
+ * reported as for spec_cycle_kb. */
+spec_status spec_decode_loop(const spec_params *p, int32_t n_cycles, const void *base,
+                             const void *target, const float *conf, float conf_threshold,
+                             const int32_t *verify_len, const void *U, const void *W,
+                             const int32_t *last_token, int32_t *draft, int32_t *out, int32_t *tau,
+                             float *p_draft, float *q_draft, int32_t *next_token, void *workspace,
+                             spec_stream_t stream);
+
 /* spec_cycle without a workspace argument, for callers that cannot allocate
  * device memory when they run a cycle (code whose allocations all belong to a
  * framework pool, a host thread that must not call cudaMalloc because it

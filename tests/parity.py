@@ -85,3 +85,37 @@ def check_invariants(out, tau, draft, K):
         assert out[b, t - 1] >= 0
         if t <= K:
             assert out[b, t - 1] != draft[b, t - 1]
+
+
+def flagged_rows(orc: dict, K: int) -> np.ndarray:
+    """Rows whose outcome depends on a flagged decision (compare_cycle's rule)."""
+    fd, fa = orc["flag_draft"].astype(int), orc["flag_accept"].astype(int)
+    stop = orc["tau"].astype(int) - 1
+    return (np.minimum(fd, fa) <= np.minimum(stop, K - 1)) | (orc["flag_final"] != 0)
+
+
+_KEYS = ("draft", "out", "tau", "p_draft", "q_draft")
+_FLAGS = ("flag_draft", "flag_accept", "flag_final")
+
+
+def compare_loop(gpu: dict, orc: dict, K: int, check_probs=True):
+    """Per-cycle comparison of a decode loop ([C, B, ...] arrays).  A row stays
+    compared while its inputs agree: once its last emitted token of a cycle
+    differs from the oracle's (allowed only after a flagged decision), the
+    next cycle starts from another token and the row leaves the comparison.
+    Returns (rows with a flagged decision summed over cycles, rows still in
+    step after the last cycle)."""
+    C, B = orc["tau"].shape
+    sync = np.ones(B, bool)
+    flagged = 0
+    for c in range(C):
+        rows = np.nonzero(sync)[0]
+        gi = {k: gpu[k][c][rows] for k in _KEYS}
+        oi = {k: orc[k][c][rows] for k in _KEYS + _FLAGS}
+        flagged += compare_cycle(gi, oi, K, rows=rows, check_probs=check_probs)
+        gl = gi["out"][np.arange(len(rows)), gi["tau"] - 1]
+        ol = oi["out"][np.arange(len(rows)), oi["tau"] - 1]
+        diff = gl != ol
+        assert np.all(flagged_rows(oi, K)[diff]), (c, rows[diff & ~flagged_rows(oi, K)])
+        sync[rows[diff]] = False
+    return flagged, sync

@@ -135,3 +135,52 @@ def test_valid_params_pass_host_validation():
         rc = L.spec_cycle(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, None,
                           None, fake, None)
         assert rc not in (sd.SPEC_ERR_INVALID_ARG, sd.SPEC_ERR_UNSUPPORTED), (kw, rc)
+
+
+def _loop_call(p, n_cycles, conf=None, vlen=None, next_token=True, nulls=()):
+    L = sd.lib()
+    fake = ctypes.c_void_p(0x1000)
+    args = dict(base=fake, target=fake, conf=conf, vlen=vlen, U=fake, W=fake, last=fake,
+                draft=None, out=fake, tau=fake, pd=None, qd=None,
+                nt=fake if next_token else None, ws=ctypes.c_void_p(0x10000))
+    for k in nulls:
+        args[k] = None
+    return L.spec_decode_loop(ctypes.byref(p.c()), n_cycles, args["base"], args["target"],
+                              args["conf"], ctypes.c_float(0.5), args["vlen"], args["U"],
+                              args["W"], args["last"], args["draft"], args["out"], args["tau"],
+                              args["pd"], args["qd"], args["nt"], args["ws"], None)
+
+
+@pytest.mark.parametrize("case", ["zero_cycles", "too_many_cycles", "no_next_token",
+                                  "conf_and_vlen", "no_target", "no_last_token", "bad_params"])
+def test_decode_loop_host_validation(case):
+    """spec_decode_loop rejects bad arguments on the host, before any launch."""
+    fake = ctypes.c_void_p(0x2000)
+    p = _p(r=64)
+    kw = {}
+    n = 3
+    if case == "zero_cycles":
+        n = 0
+    elif case == "too_many_cycles":
+        n = (1 << 16) + 1
+    elif case == "no_next_token":
+        kw = dict(next_token=False)
+    elif case == "conf_and_vlen":
+        kw = dict(conf=fake, vlen=fake)
+    elif case == "no_target":
+        kw = dict(nulls=("target",))
+    elif case == "no_last_token":
+        kw = dict(nulls=("last",))
+    elif case == "bad_params":
+        p = _p(B=0, r=64)
+    assert _loop_call(p, n, **kw) == sd.SPEC_ERR_INVALID_ARG
+
+
+def test_decode_loop_one_cycle_needs_no_next_token():
+    """One cycle carries nothing over: next_token may be NULL (the call passes
+    host validation and fails only for want of a GPU, or launches)."""
+    import torch
+    if torch.cuda.is_available():
+        return  # a fake pointer would reach the device
+    rc = _loop_call(_p(r=64), 1, next_token=False)
+    assert rc not in (sd.SPEC_ERR_INVALID_ARG, sd.SPEC_ERR_UNSUPPORTED), rc

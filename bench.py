@@ -233,7 +233,7 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     import synth
-    w = synth.WORKLOADS[WORKLOAD]
+    w = synth.WORKLOADS[args.workload]
     d = synth.make(w)
     import oracle
     oracle.build()
@@ -259,11 +259,12 @@ def run_reference(args, rank, world):
     threads = rows(args.steps, 1000)
     dt = time.perf_counter() - t0
     value = w.K * args.steps / dt
-    line = {"metric": METRIC, "value": value, "unit": "positions/s", "n_gpus": world,
+    line = {"metric": metric_name(args.workload, "cycle", 1), "value": value,
+            "unit": "positions/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "B=64 K=16 V=129280 r=256 bf16 logits, T=1.0, target noise sigma=0.5",
+            "config": {"workload": WORKLOAD_TEXT[args.workload], "call": CALL_TEXT["cycle"],
                        "sample_rows_per_step": 1, "rows_per_oracle_call": chunk,
                        "parallelism": "host cores"},
             "impl": "reference",
@@ -276,6 +277,49 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+WORKLOAD_TEXT = {
+    "c3": "B=64 K=16 V=129280 r=256 bf16 logits, T=1.0, target noise sigma=0.5",
+    "c4": "B=256 K=8 V=151936 r=256 bf16 logits, T=1.0, target noise sigma=0.5",
+    "c5": "B=128 K=32 V=129280 r=256 bf16 logits, T=1.0, target noise sigma 0.2..1.5 over rows",
+}
+
+CALL_TEXT = {
+    "cycle": "spec_cycle: drafting and verification fused in one persistent launch per cycle",
+    "loop": "spec_decode_loop: C chained cycles per persistent launch",
+    "verify": "spec_verify_block: verification of given drafts (draft logits and tokens as inputs)",
+    "draft": "spec_markov_bias_sample: sequential Markov-biased drafting only",
+}
+
+
+def metric_name(workload, call, cycles):
+    if workload == WORKLOAD and call == "cycle":
+        return METRIC
+    w = {"c3": "B=64 K=16 V=129280", "c4": "B=256 K=8 V=151936",
+         "c5": "B=128 K=32 V=129280"}[workload]
+    what = {"cycle": "draft+verify positions/sec", "loop": f"draft+verify positions/sec ({cycles} chained cycles per launch)",
+            "verify": "verified positions/sec", "draft": "drafted positions/sec"}[call]
+    return f"{what} and HBM GB/s vs B200 peak at {w}"
+
+
+def draft_only_bytes(w) -> int:
+    """Bytes of the draft-only call: every base logit row, W once, the U rows."""
+    s = 2 if w.dtype == "bf16" else 4
+    return s * w.B * w.K * w.V + s * w.r * w.V + s * w.B * w.K * w.r
+
+
+def verify_bytes(w, tau) -> float:
+    """Bytes the verification of one batch must read with the early exit: a row
+    stopping at position j (tau = j + 1) needs draft and target rows 0..j (the
+    stop row twice: statistics, then the residual draw); a row accepting all K
+    needs draft rows 0..K-1 and target rows 0..K."""
+    s = 2 if w.dtype == "bf16" else 4
+    rows = 0.0
+    for t in tau:
+        t = int(t)
+        rows += (2 * w.K + 1) if t == w.K + 1 else (2 * t + 2)
+    return s * rows * w.V
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import synth
@@ -285,30 +329,61 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     multi = shard.init("nccl", timeout_s=120)
-    w = synth.WORKLOADS[WORKLOAD]
+    w = synth.WORKLOADS[args.workload]
+    call, C = args.call, (args.cycles if args.call == "loop" else 1)
     # Weak scaling: the job's batch is world x B rows; rank r holds rows
     # [r*B, (r+1)*B) (its own seeded logits) and draws with row_offset r*B.
     row0, row1 = shard.shard_range(w.B * world, world, rank)
-    d = synth.make(w, seed=w.seed + 1000 * rank)
+    if call == "loop":
+        d = synth.make_loop(w, C, seed=w.seed + 1000 * rank)
+    else:
+        d = synth.make(w, seed=w.seed + 1000 * rank)
     dev = torch.device("cuda", local_rank)
     dd = {k: v.to(dev) for k, v in d.items()}
     p = sd.Params(B=row1 - row0, K=w.K, V=w.V, r=w.r, dtype=w.dtype, temperature=w.temperature,
                   seed=w.seed, cycle=0, row_offset=row0)
     ws = sd.make_workspace(p)
-    o = sd.alloc_outputs(p)
+    o = sd.alloc_outputs(p, n_cycles=C if call == "loop" else None)
     stream = torch.cuda.current_stream()
-
-    tau_all = torch.empty((max(1, args.steps), p.B), dtype=torch.int32, device=dev)
+    nt = torch.empty(p.B, dtype=torch.int32, device=dev)
+    if call == "verify":
+        # inputs of the verification: draft tokens and their (biased) draft
+        # logits, made once by the library's drafting call (untimed setup)
+        biased = torch.empty((p.B, w.K, w.V), dtype=torch.float32, device=dev)
+        sd.markov_bias_sample(p, dd["base"], dd["U"], dd["W"], dd["last_token"], o["draft"],
+                              None, biased, ws)
+        dd["draft_logits"] = biased.to(torch.bfloat16)
+        dd["draft"] = o["draft"].clone()
+        del biased
+        if sd.sync_status(ws) != sd.SPEC_OK:
+            raise RuntimeError("drafting for the verify inputs failed")
+    tau_shape = (C, p.B) if call == "loop" else (p.B,)
+    tau_all = torch.zeros((max(1, args.steps),) + tau_shape, dtype=torch.int32, device=dev)
 
     def step(c, tau=None):
-        p.cycle = c
-        sd.cycle(p, dd["base"], dd["target"], dd["U"], dd["W"], dd["last_token"], o["draft"],
-                 o["out"], o["tau"] if tau is None else tau, o["p_draft"], o["q_draft"], ws)
+        tau = o["tau"] if tau is None else tau
+        if call == "cycle":
+            p.cycle = c
+            sd.cycle(p, dd["base"], dd["target"], dd["U"], dd["W"], dd["last_token"], o["draft"],
+                     o["out"], tau, o["p_draft"], o["q_draft"], ws)
+        elif call == "loop":
+            p.cycle = c * C
+            sd.decode_loop(p, C, dd["base"], dd["target"], dd["U"], dd["W"], dd["last_token"],
+                           o["draft"], o["out"], tau, o["p_draft"], o["q_draft"], nt, ws,
+                           conf=dd["conf"], conf_threshold=args.conf_threshold)
+        elif call == "verify":
+            p.cycle = c
+            sd.verify_block(p, dd["target"], dd["draft_logits"], dd["draft"], o["out"], tau,
+                            o["p_draft"], o["q_draft"], ws)
+        else:
+            p.cycle = c
+            sd.markov_bias_sample(p, dd["base"], dd["U"], dd["W"], dd["last_token"], o["draft"],
+                                  o["q_draft"], None, ws)
 
     barrier = shard.barrier
 
     with ClockSampler(local_rank) as clk:
-        step(0)  # cycle 0: its outputs are compared with the oracle's sample below
+        step(0)  # the first cycle: its outputs are compared with the oracle's sample below
         out0, tau0 = o["out"].cpu().numpy(), o["tau"].cpu().numpy()
         for c in range(1, args.warmup):
             step(c)
@@ -327,32 +402,32 @@ def run_ours(args, rank, world, local_rank):
         clk.mark_end()
         barrier()
     ms = e0.elapsed_time(e1)
-    launches = args.steps  # one fused kernel per cycle
+    launches = args.steps * sd.last_launch_count()
     st = sd.sync_status(ws)
     if st != sd.SPEC_OK:
         raise RuntimeError(f"device status {sd.status_string(st)}")
-    tau = tau_all.cpu().numpy()  # every timed cycle
+    tau = tau_all.cpu().numpy().reshape(-1, p.B)  # every timed cycle
     ms_max = shard.max_over_ranks(ms)
     per_step_ms = ms_max / args.steps
-    positions = shard.sum_over_ranks(p.B * w.K * args.steps)
+    per_step = p.B * w.K * C
+    positions = shard.sum_over_ranks(per_step * args.steps)
     value = positions / (ms_max / 1e3)
 
     # end to end through the C-ABI with host buffers: pinned H2D of the step's
-    # logits and last token, the fused call, D2H of the emitted tokens and tau
-    hbase = d["base"].pin_memory()
-    htarget = d["target"].pin_memory()
-    hlast = d["last_token"].pin_memory()
-    hout = torch.empty_like(o["out"], device="cpu").pin_memory()
-    htau = torch.empty_like(o["tau"], device="cpu").pin_memory()
+    # inputs, the call, D2H of the emitted tokens and tau
+    ins = {"cycle": ("base", "target", "last_token"), "loop": ("base", "target", "last_token", "conf"),
+           "verify": ("target", "draft_logits", "draft"), "draft": ("base", "last_token")}[call]
+    outs = ("draft",) if call == "draft" else ("out", "tau")
+    hin = {k: dd[k].cpu().pin_memory() for k in ins}
+    hout = {k: torch.empty_like(o[k], device="cpu").pin_memory() for k in outs}
     e2e_steps = 20
 
     def e2e_step(c):
-        dd["base"].copy_(hbase, non_blocking=True)
-        dd["target"].copy_(htarget, non_blocking=True)
-        dd["last_token"].copy_(hlast, non_blocking=True)
+        for k in ins:
+            dd[k].copy_(hin[k], non_blocking=True)
         step(c)
-        hout.copy_(o["out"], non_blocking=True)
-        htau.copy_(o["tau"], non_blocking=True)
+        for k in outs:
+            hout[k].copy_(o[k], non_blocking=True)
 
     e2e_step(0)
     torch.cuda.synchronize()
@@ -364,48 +439,65 @@ def run_ours(args, rank, world, local_rank):
     f1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = shard.max_over_ranks(f0.elapsed_time(f1))
-    e2e_value = shard.sum_over_ranks(p.B * w.K * e2e_steps) / (e2e_ms / 1e3)
-    h2d = hbase.numel() * hbase.element_size() + htarget.numel() * htarget.element_size() + \
-        hlast.numel() * hlast.element_size()
-    d2h = hout.numel() * hout.element_size() + htau.numel() * htau.element_size()
+    e2e_value = shard.sum_over_ranks(per_step * e2e_steps) / (e2e_ms / 1e3)
+    h2d = sum(t.numel() * t.element_size() for t in hin.values())
+    d2h = sum(t.numel() * t.element_size() for t in hout.values())
 
     if rank == 0:
         peak, peak_kind = measured_peak()
-        fb = full_stream_bytes(w)
-        eb = sum(early_exit_bytes(w, t) for t in tau) / len(tau)
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
-        wl2 = w_l2_bytes(w, sms)
+        if call in ("cycle", "loop"):
+            fb = full_stream_bytes(w) * C
+            eb = sum(early_exit_bytes(w, t) for t in tau) / len(tau) * C
+            wl2 = w_l2_bytes(w, sms) * C
+            kernel = "k_cycle_tc (fused persistent draft+verify, tensor-core path)"
+        elif call == "verify":
+            fb = 2 * w.B * (2 * w.K + 1) * w.V  # every draft and target row
+            eb = sum(verify_bytes(w, t) for t in tau) / len(tau)
+            wl2 = 0
+            kernel = "verify kernels (spec_verify_block)"
+        else:
+            fb = eb = draft_only_bytes(w)
+            wl2 = w_l2_bytes(w, sms, greedy=True)
+            kernel = "draft kernel (spec_markov_bias_sample)"
         h = csrc_hash()
-        achieved = fb / (per_step_ms / 1e3) / 1e9  # GB/s, one launch per step
+        achieved = fb / (per_step_ms / 1e3) / 1e9  # GB/s over the step
+        cfg = {"workload": WORKLOAD_TEXT[args.workload], "call": CALL_TEXT[call],
+               "global_batch": w.B * world, "K": w.K, "V": w.V, "r": w.r,
+               "parallelism": f"batch-sharded x{world} (independent rows, no collective)",
+               "l2": "logit inputs > L2 (no flush between steps); W^T of 3 of each CTA's "
+                     "128-token chunks held in tensor memory, the rest streamed from L2"}
+        if call == "loop":
+            cfg.update({"cycles_per_launch": C, "conf_threshold": args.conf_threshold,
+                        "conf": "uniform(0.5, 1.0) per position (stand-in scores)"})
+        if call != "draft":
+            cfg.update({"mean_tau": float(tau.mean()), "tau_cycles": int(tau.shape[0]),
+                        "emitted_tokens_per_s": float(tau.sum()) / args.steps / (per_step_ms / 1e3)})
         line = {
-            "metric": METRIC, "value": value, "unit": "positions/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded generator: N(0,2) + Zipf(1.1) prior, target = draft + N(0,0.5), U,W ~ N(0,0.02))",
-            "config": {"workload": "B=64 K=16 V=129280 r=256 bf16 logits, T=1.0, target noise sigma=0.5",
-                       "global_batch": w.B * world, "K": w.K, "V": w.V, "r": w.r,
-                       "parallelism": f"batch-sharded x{world} (independent rows, no collective)",
-                       "l2": "logit inputs 546 MB > L2 (no flush between cycles); W^T of 3 of each "
-                             "CTA's 128-token chunks held in tensor memory, the rest streamed from L2",
-                       "mean_tau": float(tau.mean()), "tau_cycles": int(tau.shape[0]),
-                       "emitted_tokens_per_s": float(tau.sum()) / tau.shape[0] / (per_step_ms / 1e3)},
+            "metric": metric_name(args.workload, call, C), "value": value, "unit": "positions/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": per_step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded generator: N(0,2) + Zipf(1.1) prior, target = draft + N(0,sigma), U,W ~ N(0,0.02))",
+            "config": cfg,
             "gpu_launches": launches * world,
             "rows_per_rank": p.B,
             "hbm_gbs_full_stream": achieved,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": recorded_traffic(h),
+                         "frac": achieved / peak,
+                         "traffic": recorded_traffic(h) if (call == "cycle" and args.workload == WORKLOAD) else None,
                          "peak_kind": peak_kind,
                          "bytes_per_launch": fb, "early_exit_bytes_per_launch": eb,
                          "early_exit_achieved": eb / (per_step_ms / 1e3) / 1e9,
                          "frac_vs_nominal_8000": achieved / 8000.0,
                          "w_from_l2_bytes_per_launch": wl2,
                          "w_from_l2_achieved_gbs": wl2 / (per_step_ms / 1e3) / 1e9,
-                         "kernel": "k_cycle_tc (fused persistent draft+verify, tensor-core path)"},
+                         "kernel": kernel},
             "clocks": clk.summary(),
             "e2e": {"value": e2e_value, "unit": "positions/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
         }
-        if world == 1:
+        if world == 1 and call == "cycle":
             if args.no_cpu_baseline:
                 line["cpu_baseline"] = None
             else:
@@ -427,6 +519,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the timed oracle sample (profiling runs)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WORKLOAD_TEXT),
+                    help="c3 is the headline configuration")
+    ap.add_argument("--call", default="cycle", choices=sorted(CALL_TEXT),
+                    help="which entry point one step runs (cycle: the headline)")
+    ap.add_argument("--cycles", type=int, default=4, help="cycles per launch for --call loop")
+    ap.add_argument("--conf-threshold", type=float, default=0.0,
+                    help="prefix-survival threshold for --call loop (0: every K_b = K)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -28,6 +28,7 @@ _SIGS = {
     "spec_markov_bias": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P]),
     "spec_markov_bias_sample": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_verify_block": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "spec_verify_block_kb": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_cycle": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_cycle_kb": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_decode_loop": (ctypes.c_int, [_P, ctypes.c_int32, _P, _P, _P, ctypes.c_float, _P, _P, _P,
@@ -159,6 +160,15 @@ def verify_block(p: Params, target, draft_logits, draft, out, tau, p_draft, q_dr
     _check(lib().spec_verify_block(ctypes.byref(p.c()), _ptr(target), _ptr(draft_logits),
                                    _ptr(draft), _ptr(out), _ptr(tau), _ptr(p_draft),
                                    _ptr(q_draft), _ptr(ws), _stream(stream)), "spec_verify_block")
+
+
+def verify_block_kb(p: Params, target, draft_logits, draft, verify_len, out, tau, p_draft, q_draft,
+                    ws, stream=None):
+    """spec_verify_block_kb: verification with a verify length K_b per row."""
+    _check(lib().spec_verify_block_kb(ctypes.byref(p.c()), _ptr(target), _ptr(draft_logits),
+                                      _ptr(draft), _ptr(verify_len), _ptr(out), _ptr(tau),
+                                      _ptr(p_draft), _ptr(q_draft), _ptr(ws), _stream(stream)),
+           "spec_verify_block_kb")
 
 
 def cycle(p: Params, base, target, U, W, last_token, draft, out, tau, p_draft, q_draft, ws,

@@ -142,6 +142,25 @@ cudaError_t launch_debug_curand_philox(const uint32_t* ctr, const uint32_t* key,
   return cudaGetLastError();
 }
 
+template <typename T, typename TD>
+cudaError_t verify_dispatch(const spec_params* p, const void* target,
+                                   const void* draft_logits, const int32_t* draft,
+                                   const int32_t* vlen, int32_t* out, int32_t* tau, float* p_draft,
+                                   float* q_draft, bool fused, uint8_t* body, WsHeader* h, int sms,
+                                   cudaStream_t st, int* launches) {
+  const int gr = p->greedy ? 1 : 0;
+  if (fused) {
+    *launches = 1;
+    return launch_verify_ee((const T*)target, (const TD*)draft_logits, draft, vlen, out, tau,
+                            p_draft, q_draft, p->B, p->K, p->V, p->temperature, gr, p->seed,
+                            p->cycle, p->row_offset, spin_of(p), (p->flags & SPEC_FLAG_TRACE) != 0,
+                            body, h, sms, st);
+  }
+  return launch_verify((const T*)target, (const TD*)draft_logits, draft, out, tau, p_draft,
+                       q_draft, p->B, p->K, p->V, p->temperature, gr, p->seed, p->cycle,
+                       p->row_offset, body, h, sms, st, launches);
+}
+
 }  // namespace specdec
 
 using namespace specdec;
@@ -167,7 +186,7 @@ size_t spec_workspace_size(const spec_params* p) {
   if (check_params(p) != SPEC_OK) return 0;
   const int sms = num_sms();
   if (sms <= 0) return 0;
-  size_t need = verify_ws_bytes(p->B, p->K, p->V);
+  size_t need = std::max(verify_ws_bytes(p->B, p->K, p->V), verify_ee_ws_bytes(p->B, p->V, sms));
   CycleGeom g;
   const char* why = nullptr;
   if (cycle_geometry(p->B, p->K, p->V, p->r, p->dtype, p->flags, sms, &g, &why))
@@ -408,9 +427,10 @@ spec_status spec_decode_loop(const spec_params* p, int32_t n_cycles, const void*
                       q_draft, ws, stream, loop);
 }
 
-spec_status spec_verify_block(const spec_params* p, const void* target, const void* draft_logits,
-                              const int32_t* draft, int32_t* out, int32_t* tau, float* p_draft,
-                              float* q_draft, void* ws, spec_stream_t stream) {
+static spec_status run_verify(const spec_params* p, const void* target, const void* draft_logits,
+                              const int32_t* draft, const int32_t* vlen, int32_t* out,
+                              int32_t* tau, float* p_draft, float* q_draft, void* ws,
+                              spec_stream_t stream) {
   g_last_launches = 0;
   spec_status s = check_params(p);
   if (s != SPEC_OK) return s;
@@ -420,30 +440,54 @@ spec_status spec_verify_block(const spec_params* p, const void* target, const vo
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SPEC_ERR_WORKSPACE;
   const int sms = num_sms();
   if (sms <= 0) return SPEC_ERR_CUDA;
+  VerifyGeom vg;
+  const bool fused = verify_ee_geometry(p->B, p->V, sms, p->dtype == SPEC_BF16 ? 2 : 4,
+                                        p->draft_dtype == SPEC_BF16 ? 2 : 4, p->greedy ? 1 : 0, &vg);
+  if (vlen && !fused) {
+    fprintf(stderr, "specdec: per-row verify lengths need the one-launch verification (B <= 4096 "
+                    "and a vocabulary slice per SM that fits its shared-memory ring)\n");
+    return SPEC_ERR_UNSUPPORTED;
+  }
   int launches = 0;
   cudaError_t e;
   cudaStream_t st = (cudaStream_t)stream;
-  const int B = p->B, K = p->K, V = p->V, gr = p->greedy ? 1 : 0;
   WsHeader* h = header_of(ws);
   uint8_t* body = body_of(ws);
   if (p->dtype == SPEC_BF16 && p->draft_dtype == SPEC_BF16)
-    e = launch_verify((const __nv_bfloat16*)target, (const __nv_bfloat16*)draft_logits, draft, out,
-                      tau, p_draft, q_draft, B, K, V, p->temperature, gr, p->seed, p->cycle, p->row_offset, body,
-                      h, sms, st, &launches);
+    e = verify_dispatch<__nv_bfloat16, __nv_bfloat16>(p, target, draft_logits, draft, vlen, out, tau,
+                                                      p_draft, q_draft, fused, body, h, sms, st,
+                                                      &launches);
   else if (p->dtype == SPEC_BF16)
-    e = launch_verify((const __nv_bfloat16*)target, (const float*)draft_logits, draft, out, tau,
-                      p_draft, q_draft, B, K, V, p->temperature, gr, p->seed, p->cycle, p->row_offset, body, h,
-                      sms, st, &launches);
+    e = verify_dispatch<__nv_bfloat16, float>(p, target, draft_logits, draft, vlen, out, tau,
+                                              p_draft, q_draft, fused, body, h, sms, st, &launches);
   else if (p->draft_dtype == SPEC_BF16)
-    e = launch_verify((const float*)target, (const __nv_bfloat16*)draft_logits, draft, out, tau,
-                      p_draft, q_draft, B, K, V, p->temperature, gr, p->seed, p->cycle, p->row_offset, body, h,
-                      sms, st, &launches);
+    e = verify_dispatch<float, __nv_bfloat16>(p, target, draft_logits, draft, vlen, out, tau,
+                                              p_draft, q_draft, fused, body, h, sms, st, &launches);
   else
-    e = launch_verify((const float*)target, (const float*)draft_logits, draft, out, tau, p_draft,
-                      q_draft, B, K, V, p->temperature, gr, p->seed, p->cycle, p->row_offset, body, h, sms, st,
-                      &launches);
+    e = verify_dispatch<float, float>(p, target, draft_logits, draft, vlen, out, tau, p_draft,
+                                      q_draft, fused, body, h, sms, st, &launches);
   g_last_launches = launches;
-  return e == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
+  if (e != cudaSuccess) {
+    fprintf(stderr, "specdec: launch failed: %s\n", cudaGetErrorString(e));
+    return SPEC_ERR_CUDA;
+  }
+  return SPEC_OK;
+}
+
+spec_status spec_verify_block(const spec_params* p, const void* target, const void* draft_logits,
+                              const int32_t* draft, int32_t* out, int32_t* tau, float* p_draft,
+                              float* q_draft, void* ws, spec_stream_t stream) {
+  return run_verify(p, target, draft_logits, draft, nullptr, out, tau, p_draft, q_draft, ws,
+                    stream);
+}
+
+spec_status spec_verify_block_kb(const spec_params* p, const void* target,
+                                 const void* draft_logits, const int32_t* draft,
+                                 const int32_t* verify_len, int32_t* out, int32_t* tau,
+                                 float* p_draft, float* q_draft, void* ws, spec_stream_t stream) {
+  if (!verify_len) return SPEC_ERR_INVALID_ARG;
+  return run_verify(p, target, draft_logits, draft, verify_len, out, tau, p_draft, q_draft, ws,
+                    stream);
 }
 
 spec_status spec_l2_persist(const void* ptr, size_t bytes, spec_stream_t stream) {

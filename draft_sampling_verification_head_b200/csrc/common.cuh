@@ -365,6 +365,13 @@ SPEC_DEV bool grid_wait_count(WsHeader* h, const uint32_t* counter, uint32_t tar
   return false;
 }
 
+// Device clock in nanoseconds (timelines of the trace flag).
+SPEC_DEV uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
 SPEC_DEV float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

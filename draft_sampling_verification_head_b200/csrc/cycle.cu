@@ -166,12 +166,6 @@ __host__ __device__ inline size_t bucket_region_bytes(int nc, int N) {
 
 SPEC_DEV void named_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
-SPEC_DEV uint64_t globaltimer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
 // Eight consecutive logits as raw 16-byte loads (streaming, L1 bypass).
 template <typename T>
 struct Raw8;

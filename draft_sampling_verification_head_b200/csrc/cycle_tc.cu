@@ -158,12 +158,6 @@ SPEC_DEV RecT load_rec(const RecT* src) {
 SPEC_DEV void named_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 SPEC_DEV void quartet_sync(int q) { asm volatile("bar.sync %0, 128;" ::"r"(2 + q) : "memory"); }
 
-SPEC_DEV uint64_t globaltimer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
 // D[tmem] (+)= A[tmem] * B[smem], kind::f16 (bf16 inputs, fp32 accumulate)
 SPEC_DEV void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                            uint32_t accumulate) {

@@ -39,6 +39,24 @@ cudaError_t launch_verify(const T* target, const TD* draft_logits, const int32_t
                           uint64_t cycle, uint32_t row0, uint8_t* ws_body, WsHeader* hdr, int num_sms,
                           cudaStream_t st, int* launches);
 
+// One persistent launch with early exit (rows up to 4096, slices whose ring
+// fits shared memory); geometry false otherwise.
+struct VerifyGeom {
+  int G, seg;          // CTAs, tokens per CTA slice
+  int S, slotb, doff;  // ring slots per warp, slot bytes, draft offset in a slot
+  size_t smem;         // dynamic shared memory
+};
+bool verify_ee_geometry(int B, int V, int num_sms, int tsize, int dsize, int greedy,
+                        VerifyGeom* g);
+size_t verify_ee_ws_bytes(int B, int V, int num_sms);
+template <typename T, typename TD>
+cudaError_t launch_verify_ee(const T* target, const TD* draft_logits, const int32_t* draft,
+                             const int32_t* vlen, int32_t* out, int32_t* tau, float* p_draft,
+                             float* q_draft, int B, int K, int V, float temperature, int greedy,
+                             uint64_t seed, uint64_t cycle, uint32_t row0, uint64_t spin,
+                             bool trace, uint8_t* body, WsHeader* hdr, int num_sms,
+                             cudaStream_t st);
+
 // ---- Fused persistent draft (+ verify) ---------------------------------------
 enum CycleMode : int32_t { MODE_CYCLE = 0, MODE_DRAFT = 1 };
 

@@ -132,10 +132,29 @@ spec_status spec_markov_bias_sample(const spec_params *p, const void *base, cons
 /* Verification of given drafts against the target rows (section "Jak działa
  * spekulatywne dekodowanie"): draft_logits [B, K, V] are the final (biased)
  * draft logits in draft_dtype, draft [B, K] the tokens drawn from them.
- * p_draft and q_draft may be NULL. */
+ * One persistent launch with early exit (B <= 4096 and V up to 2048 tokens
+ * per SM): positions are decided a few at a time, and the draft and target
+ * rows of a position past a row's first rejection are never read.  So
+ * q_draft[b, i] is written for the positions whose accept test ran (NaN
+ * after), like p_draft.  Larger shapes take a multi-launch path that reads
+ * every row and writes q_draft for all K positions.  p_draft and q_draft may
+ * be NULL. */
 spec_status spec_verify_block(const spec_params *p, const void *target, const void *draft_logits,
                               const int32_t *draft, int32_t *out, int32_t *tau, float *p_draft,
                               float *q_draft, void *workspace, spec_stream_t stream);
+
+/* spec_verify_block with a verify length per request (the scheduler's K_b,
+ * section "Optymalizacja weryfikacji i wydajności"): verify_len [B] int32
+ * (device), K_b in 1..K.  Row b verifies positions 0..K_b-1 and draws its
+ * bonus from target row K_b, so tau_b <= K_b + 1; rows past K_b are never
+ * read.  A K_b outside 1..K is clamped and reported as SPEC_ERR_INVALID_ARG by
+ * spec_sync_status.  Shapes the one-launch path does not take return
+ * SPEC_ERR_UNSUPPORTED. */
+spec_status spec_verify_block_kb(const spec_params *p, const void *target,
+                                 const void *draft_logits, const int32_t *draft,
+                                 const int32_t *verify_len, int32_t *out, int32_t *tau,
+                                 float *p_draft, float *q_draft, void *workspace,
+                                 spec_stream_t stream);
 
 /* One whole cycle: drafting and verification fused in one persistent launch
  * (target rows are read only up to each row's first rejection).  draft,

@@ -119,3 +119,16 @@ def compare_loop(gpu: dict, orc: dict, K: int, check_probs=True):
         assert np.all(flagged_rows(oi, K)[diff]), (c, rows[diff & ~flagged_rows(oi, K)])
         sync[rows[diff]] = False
     return flagged, sync
+
+
+def early_exit_q(gpu: dict, orc: dict):
+    """Verification with early exit reports q_i(d_i) only where the accept test
+    ran (positions up to the row's stop, NaN after); the oracle defines it at
+    every position.  Checks the GPU's NaN tail, then keeps q up to the earlier
+    of the two stops on both sides for compare_cycle."""
+    for b in range(len(orc["tau"])):
+        sg, so = int(gpu["tau"][b]) - 1, int(orc["tau"][b]) - 1
+        assert np.all(np.isnan(gpu["q_draft"][b, sg + 1:])), (b, gpu["q_draft"][b])
+        m = min(sg, so)
+        gpu["q_draft"][b, m + 1:] = np.nan
+        orc["q_draft"][b, m + 1:] = np.nan

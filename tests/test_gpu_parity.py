@@ -14,7 +14,7 @@ from scipy import stats
 import oracle
 import synth
 from oracle import exact_law as EL
-from parity import check_invariants, compare_cycle, compare_draft, note_near
+from parity import check_invariants, compare_cycle, compare_draft, note_near, early_exit_q
 
 import draft_sampling_verification_head_b200 as sd
 
@@ -177,6 +177,7 @@ def test_verify_block_vs_oracle(B, K, V, dtype, ddtype, greedy):
     gpu["draft"] = drafts
     o["draft"] = drafts
     o["flag_draft"] = np.full(B, K, np.int32)
+    early_exit_q(gpu, o)
     compare_cycle(gpu, o, K)
     check_invariants(gpu["out"], gpu["tau"], drafts, K)
 
@@ -280,6 +281,7 @@ def test_verify_block_row_offset():
     ref = {k: (v[b0:] if isinstance(v, np.ndarray) else v) for k, v in o.items()}
     ref["draft"] = drafts[b0:]
     ref["flag_draft"] = np.full(B - b0, K, np.int32)
+    early_exit_q(gpu, ref)
     compare_cycle(gpu, ref, K)
 
 

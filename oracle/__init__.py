@@ -43,7 +43,7 @@ class _Params(ctypes.Structure):
                 ("r", ctypes.c_int32), ("dtype", ctypes.c_int32), ("draft_dtype", ctypes.c_int32),
                 ("temperature", ctypes.c_double), ("greedy", ctypes.c_int32),
                 ("seed", ctypes.c_uint64), ("cycle", ctypes.c_uint64),
-                ("verify_len", ctypes.c_void_p)]
+                ("verify_len", ctypes.c_void_p), ("Wh", ctypes.c_void_p)]
 
 
 class _Outputs(ctypes.Structure):
@@ -96,6 +96,7 @@ class Params:
     cycle: int = 0
     draft_dtype: str | None = None  # verify-only: dtype of the given draft logits
     verify_len: np.ndarray | None = None  # [B] int32 per-row verify length K_b (1..K), or None
+    Wh: np.ndarray | None = None  # [r, r] RNN head weights (raw storage of dtype), or None (Markov)
 
     def c(self) -> _Params:
         dd = self.draft_dtype or self.dtype
@@ -105,9 +106,14 @@ class Params:
         if self.verify_len is not None:
             self._vl = np.ascontiguousarray(self.verify_len, dtype=np.int32)  # kept alive
             vl = self._vl.ctypes.data_as(ctypes.c_void_p)
+        wh = None
+        if self.Wh is not None:
+            self._wh = _raw(self.Wh, self.dtype)  # kept alive
+            assert self._wh.size == self.r * self.r
+            wh = self._wh.ctypes.data_as(ctypes.c_void_p)
         return _Params(self.B, self.K, self.V, self.r, _DT[self.dtype], _DT[dd], T,
                        1 if self.greedy else 0, self.seed & (2**64 - 1), self.cycle & (2**64 - 1),
-                       vl)
+                       vl, wh)
 
 
 def _raw(a: np.ndarray, dtype: str) -> np.ndarray:

@@ -40,12 +40,25 @@ def draft_q(base, U, W, i, prev, T):
     return softmax(z, T)
 
 
-def exact_law(base, target, U, W, last_token, T, rule="standard", verify_len=None):
+def rnn_state(U, Wh, prev, s_old):
+    """RNN head state (float64): clamp(U[prev] + Wh . s_old, -1, 1); s_old None
+    at the first position.  Exact for inputs whose sums are exactly
+    representable (the pins use small dyadic values)."""
+    pre = np.asarray(U[prev], np.float64).copy()
+    if s_old is not None:
+        pre = pre + np.asarray(Wh, np.float64) @ s_old
+    return np.clip(pre, -1.0, 1.0)
+
+
+def exact_law(base, target, U, W, last_token, T, rule="standard", verify_len=None, Wh=None):
     """Return {(tau, out_tuple): probability} for one batch row.
 
     base: [K, V], target: [K+1, V], U: [V, r], W: [r, V] (float64-convertible).
     verify_len: the row's verify length K_b (1..K; default K): positions
     0..K_b-1 are drafted and verified, the bonus comes from target row K_b.
+    Wh: [r, r] recurrent weights of the RNN head (the bias of position i is
+    s_i . W with s_i = rnn_state(U, Wh, prev_i, s_{i-1})), or None for the
+    Markov head.
     """
     base = np.asarray(base, np.float64)
     target = np.asarray(target, np.float64)
@@ -55,14 +68,19 @@ def exact_law(base, target, U, W, last_token, T, rule="standard", verify_len=Non
     P = [softmax(target[i], T) for i in range(K + 1)]
     law = defaultdict(float)
 
-    def walk(i, prev, prob, prefix):
+    def walk(i, prev, prob, prefix, s_old=None):
         if prob == 0.0:
             return
         if i == K:
             for x in range(V):
                 law[(K + 1, tuple(prefix + [x]))] += prob * P[K][x]
             return
-        q = draft_q(base, U, W, i, prev, T)
+        if Wh is None:
+            q = draft_q(base, U, W, i, prev, T)
+            s_new = None
+        else:
+            s_new = rnn_state(U, Wh, prev, s_old)
+            q = softmax(np.asarray(base[i], np.float64) + s_new @ np.asarray(W, np.float64), T)
         p = P[i]
         if rule == "ratio_qp":
             acc = np.minimum(1.0, np.where(p > 0, q / np.where(p > 0, p, 1.0), 1.0))
@@ -80,7 +98,7 @@ def exact_law(base, target, U, W, last_token, T, rule="standard", verify_len=Non
             law[(i + 1, tuple(prefix + [x]))] += prob * rej_total * res[x]
         for d in range(V):
             if q[d] > 0:
-                walk(i + 1, d, prob * q[d] * acc[d], prefix + [d])
+                walk(i + 1, d, prob * q[d] * acc[d], prefix + [d], s_new)
 
     walk(0, int(last_token), 1.0, [])
     return dict(law)

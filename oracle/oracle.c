@@ -224,12 +224,55 @@ static int32_t verify_len_of(const orc_params *P, int32_t b) {
   return P->verify_len ? P->verify_len[b] : P->K;
 }
 
+/* fp32 -> bf16 -> fp32, rounding to nearest with ties to even (finite x). */
+static float round_bf16(float x) {
+  uint32_t u;
+  memcpy(&u, &x, 4);
+  u = (u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u;
+  float y;
+  memcpy(&y, &u, 4);
+  return y;
+}
+
+/* RNN head state update (orc_params.Wh): s_new from s_old (NULL at i = 0). */
+static void rnn_state(const orc_params *P, const void *U, int32_t prev, const float *s_old,
+                      float *s_new) {
+  const int32_t r = P->r;
+  for (int32_t j = 0; j < r; ++j) {
+    float acc = 0.0f;
+#if !(defined(ORC_PLANT) && ORC_PLANT == 4) /* planted mistake: the state forgets the prefix */
+    if (s_old)
+      for (int32_t k = 0; k < r; ++k)
+        acc = fmaf(s_old[k], (float)load_elem(P->Wh, P->dtype, (int64_t)j * r + k), acc);
+#endif
+    const float pre = (float)load_elem(U, P->dtype, (int64_t)prev * r + j) + acc;
+    const float h = fminf(fmaxf(pre, -1.0f), 1.0f);
+    s_new[j] = P->dtype == ORC_BF16 ? round_bf16(h) : h;
+  }
+}
+
+/* z = base[b, i, :] + s . W for an explicit head state s[r] (double). */
+static void biased_row_state(const orc_params *P, const void *base, const void *W, int32_t b,
+                             int32_t i, const float *s, double *z) {
+  const int32_t K = P->K, V = P->V, r = P->r;
+  const int64_t row = ((int64_t)b * K + i) * V;
+  for (int32_t v = 0; v < V; ++v) z[v] = 0.0;
+  for (int32_t k = 0; k < r; ++k) {
+    const double u = s[k];
+    const int64_t wrow = (int64_t)k * V;
+    for (int32_t v = 0; v < V; ++v) z[v] += u * load_elem(W, P->dtype, wrow + v);
+  }
+  for (int32_t v = 0; v < V; ++v) z[v] = load_elem(base, P->dtype, row + v) + z[v];
+}
+
 /* Draft one row: fills d[K], qd[K], zrows[K*V] (z values), flag. */
 static int draft_row(const orc_params *P, const void *base, const void *U, const void *W,
                      int32_t b, int32_t prev0, int32_t *d, double *qd, double *zrows,
                      int32_t *flag_draft, double *scratch) {
   const int32_t K = P->K, V = P->V, Kb = verify_len_of(P, b);
   int32_t prev = prev0;
+  float *st = NULL;  /* RNN head: the state of the last step and the next one */
+  if (P->Wh) st = (float *)malloc(sizeof(float) * 2 * (size_t)(P->r > 0 ? P->r : 1));
   if (flag_draft) *flag_draft = K;
   for (int32_t i = Kb; i < K; ++i) {  /* positions past the verify length are not drafted */
     d[i] = -1;
@@ -237,7 +280,13 @@ static int draft_row(const orc_params *P, const void *base, const void *U, const
   }
   for (int32_t i = 0; i < Kb; ++i) {
     double *z = zrows + (size_t)i * V;
-    biased_row(P, base, U, W, b, i, prev, z);
+    if (st) {
+      float *s_new = st + (size_t)(i & 1) * P->r, *s_old = st + (size_t)((i + 1) & 1) * P->r;
+      rnn_state(P, U, prev, i == 0 ? NULL : s_old, s_new);
+      biased_row_state(P, base, W, b, i, s_new, z);
+    } else {
+      biased_row(P, base, U, W, b, i, prev, z);
+    }
     int32_t near = 0, tok;
     if (P->greedy) {
       tok = argmax_lowest(z, V, &near, 1e-5);
@@ -258,6 +307,7 @@ static int draft_row(const orc_params *P, const void *base, const void *U, const
     prev = tok;
 #endif
   }
+  free(st);
   return 0;
 }
 

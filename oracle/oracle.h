@@ -72,6 +72,20 @@ typedef struct {
    * 0..K_b-1 only and takes its bonus from target row K_b (the rule above
    * with K_b in place of K); draft[b, i] = -1 and q_draft NaN for i >= K_b. */
   const int32_t *verify_len;
+  /* [r, r] (dtype) recurrent weights of the RNN sequential head, or NULL for
+   * the Markov head.  aigest.pl "DeepSeek prezentuje DSpark", section
+   * "Innowacje w tworzeniu tokenów": an optional RNN head tracks the whole
+   * block prefix instead of the previous token only.  The pages give no
+   * formula.  Reading (an Elman recurrence in the Markov head's factors):
+   *   s_{-1} = 0,  s_i[j] = clamp(U[prev_i, j] + sum_k Wh[j, k] s_{i-1}[k], -1, 1),
+   *   bias_i = s_i . W,
+   * prev_i as for the Markov head.  The state is the bias's low-rank operand,
+   * so it is kept in the head's dtype: in fp32 the sum runs as fmaf in
+   * ascending k from 0, the U term is added after it, the clamp is exact, and
+   * for bf16 the result is rounded to bf16 (nearest, ties to even).  Every
+   * step of this is exactly reproducible, so both sides hold the same state
+   * bit for bit. */
+  const void *Wh;
 } orc_params;
 
 /* Per-row outputs for rows [b_begin, b_end); arrays are indexed by b - b_begin.

@@ -288,6 +288,7 @@ CALL_TEXT = {
     "loop": "spec_decode_loop: C chained cycles per persistent launch",
     "verify": "spec_verify_block: verification of given drafts (draft logits and tokens as inputs)",
     "draft": "spec_markov_bias_sample: sequential Markov-biased drafting only",
+    "rnn": "spec_cycle_rnn: the fused cycle with the RNN sequential head (Wh ~ N(0, 1/r))",
 }
 
 
@@ -297,6 +298,7 @@ def metric_name(workload, call, cycles):
     w = {"c3": "B=64 K=16 V=129280", "c4": "B=256 K=8 V=151936",
          "c5": "B=128 K=32 V=129280"}[workload]
     what = {"cycle": "draft+verify positions/sec", "loop": f"draft+verify positions/sec ({cycles} chained cycles per launch)",
+            "rnn": "draft+verify positions/sec (RNN sequential head)",
             "verify": "verified positions/sec", "draft": "drafted positions/sec"}[call]
     return f"{what} and HBM GB/s vs B200 peak at {w}"
 
@@ -357,6 +359,8 @@ def run_ours(args, rank, world, local_rank):
         del biased
         if sd.sync_status(ws) != sd.SPEC_OK:
             raise RuntimeError("drafting for the verify inputs failed")
+    if call == "rnn":
+        dd["Wh"] = synth.rnn_weights(w).to(dev)
     tau_shape = (C, p.B) if call == "loop" else (p.B,)
     tau_all = torch.zeros((max(1, args.steps),) + tau_shape, dtype=torch.int32, device=dev)
 
@@ -371,6 +375,10 @@ def run_ours(args, rank, world, local_rank):
             sd.decode_loop(p, C, dd["base"], dd["target"], dd["U"], dd["W"], dd["last_token"],
                            o["draft"], o["out"], tau, o["p_draft"], o["q_draft"], nt, ws,
                            conf=dd["conf"], conf_threshold=args.conf_threshold)
+        elif call == "rnn":
+            p.cycle = c
+            sd.cycle_rnn(p, dd["base"], dd["target"], dd["U"], dd["W"], dd["Wh"], dd["last_token"],
+                         o["draft"], o["out"], tau, o["p_draft"], o["q_draft"], ws)
         elif call == "verify":
             p.cycle = c
             sd.verify_block(p, dd["target"], dd["draft_logits"], dd["draft"], o["out"], tau,
@@ -415,7 +423,8 @@ def run_ours(args, rank, world, local_rank):
 
     # end to end through the C-ABI with host buffers: pinned H2D of the step's
     # inputs, the call, D2H of the emitted tokens and tau
-    ins = {"cycle": ("base", "target", "last_token"), "loop": ("base", "target", "last_token", "conf"),
+    ins = {"cycle": ("base", "target", "last_token"), "rnn": ("base", "target", "last_token"),
+           "loop": ("base", "target", "last_token", "conf"),
            "verify": ("target", "draft_logits", "draft"), "draft": ("base", "last_token")}[call]
     outs = ("draft",) if call == "draft" else ("out", "tau")
     hin = {k: dd[k].cpu().pin_memory() for k in ins}
@@ -446,7 +455,7 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0:
         peak, peak_kind = measured_peak()
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
-        if call in ("cycle", "loop"):
+        if call in ("cycle", "loop", "rnn"):
             fb = full_stream_bytes(w) * C
             eb = sum(early_exit_bytes(w, t) for t in tau) / len(tau) * C
             wl2 = w_l2_bytes(w, sms) * C

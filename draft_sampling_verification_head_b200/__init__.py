@@ -33,6 +33,7 @@ _SIGS = {
     "spec_cycle_kb": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_decode_loop": (ctypes.c_int, [_P, ctypes.c_int32, _P, _P, _P, ctypes.c_float, _P, _P, _P,
                                          _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "spec_cycle_rnn": (ctypes.c_int, [_P] * 14),
     "spec_sync_status": (ctypes.c_int, [_P, _P]),
     "spec_cycle_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_l2_persist": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
@@ -198,6 +199,15 @@ def decode_loop(p: Params, n_cycles, base, target, U, W, last_token, draft, out,
                                   _ptr(W), _ptr(last_token), _ptr(draft), _ptr(out), _ptr(tau),
                                   _ptr(p_draft), _ptr(q_draft), _ptr(next_token), _ptr(ws),
                                   _stream(stream)), "spec_decode_loop")
+
+
+def cycle_rnn(p: Params, base, target, U, W, Wh, last_token, draft, out, tau, p_draft, q_draft, ws,
+              stream=None):
+    """spec_cycle_rnn: one cycle with the RNN sequential head (Wh [r, r] bf16)."""
+    _check(lib().spec_cycle_rnn(ctypes.byref(p.c()), _ptr(base), _ptr(target), _ptr(U), _ptr(W),
+                                _ptr(Wh), _ptr(last_token), _ptr(draft), _ptr(out), _ptr(tau),
+                                _ptr(p_draft), _ptr(q_draft), _ptr(ws), _stream(stream)),
+           "spec_cycle_rnn")
 
 
 def cycle_noalloc(p: Params, base, target, U, W, last_token, draft, out, tau, p_draft, q_draft,

@@ -192,7 +192,7 @@ size_t spec_workspace_size(const spec_params* p) {
   if (cycle_geometry(p->B, p->K, p->V, p->r, p->dtype, p->flags, sms, &g, &why))
     need = std::max(need, cycle_ws_bytes(p->K, g));
   if (cycle_tc_geometry(p->B, p->K, p->V, p->r, p->dtype, p->flags, sms, &g, &why))
-    need = std::max(need, cycle_tc_ws_bytes(p->K, g));
+    need = std::max(need, cycle_tc_ws_bytes(p->K, p->r, g));
   return round256(sizeof(WsHeader) + need);
 }
 
@@ -240,13 +240,15 @@ spec_status spec_markov_bias(const spec_params* p, const void* U, const void* W,
 }
 
 // The fused cycle on the tensor-core path (geometry already decided).
-// Loop inputs of the tensor-core cycle: cycles per launch, confidence scores
-// with their threshold, and the carried last tokens (one cycle: all unset).
+// Extra inputs of the tensor-core cycle: cycles per launch, confidence scores
+// with their threshold, the carried last tokens, the RNN head's recurrence
+// (one plain cycle of the Markov head: all unset).
 struct LoopInputs {
   int ncyc = 1;
   const float* conf = nullptr;
   float conf_thr = 0.f;
   int32_t* next_token = nullptr;
+  const void* Wh = nullptr;
 };
 
 static spec_status run_cycle_tc(const spec_params* p, const CycleGeom& g, const void* base,
@@ -269,6 +271,7 @@ static spec_status run_cycle_tc(const spec_params* p, const CycleGeom& g, const 
   L.conf_thr = loop.conf_thr;
   L.next_token = loop.next_token;
   L.ncyc = loop.ncyc;
+  L.Wh = loop.Wh;
   L.draft = draft;
   L.out = out;
   L.tau = tau;
@@ -472,6 +475,33 @@ static spec_status run_verify(const spec_params* p, const void* target, const vo
     return SPEC_ERR_CUDA;
   }
   return SPEC_OK;
+}
+
+spec_status spec_cycle_rnn(const spec_params* p, const void* base, const void* target,
+                           const void* U, const void* W, const void* Wh, const int32_t* last_token,
+                           int32_t* draft, int32_t* out, int32_t* tau, float* p_draft,
+                           float* q_draft, void* ws, spec_stream_t stream) {
+  g_last_launches = 0;
+  spec_status s = check_params(p);
+  if (s != SPEC_OK) return s;
+  if (!base || !target || !last_token || !out || !tau || !U || !W || !Wh || p->r < 1)
+    return SPEC_ERR_INVALID_ARG;
+  if (!aligned16(base) || !aligned16(target) || !aligned16(U) || !aligned16(W) || !aligned16(Wh))
+    return SPEC_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SPEC_ERR_WORKSPACE;
+  const int sms = num_sms();
+  if (sms <= 0) return SPEC_ERR_CUDA;
+  CycleGeom g;
+  const char* why = nullptr;
+  if (!cycle_tc_geometry(p->B, p->K, p->V, p->r, p->dtype, p->flags, sms, &g, &why)) {
+    fprintf(stderr, "specdec: the RNN head needs the tensor-core cycle (bf16, rank a multiple "
+                    "of 64 up to 256): %s\n", why);
+    return SPEC_ERR_UNSUPPORTED;
+  }
+  LoopInputs loop;
+  loop.Wh = Wh;
+  return run_cycle_tc(p, g, base, target, U, W, last_token, nullptr, draft, out, tau, p_draft,
+                      q_draft, ws, stream, loop);
 }
 
 spec_status spec_verify_block(const spec_params* p, const void* target, const void* draft_logits,

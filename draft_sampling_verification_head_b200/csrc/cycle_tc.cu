@@ -77,6 +77,9 @@ struct ArgsTC {
   const int32_t* vlen;   // [C][B] per-row verify length K_b (1..K), or null
   const float* conf;     // [C][B][K] confidence scores (used without vlen), or null
   int32_t* next_token;   // [B] each row's last emitted token (carried between cycles), or null
+  const __nv_bfloat16* Wh;  // [r][r] RNN head recurrence (row j: weights of s_{i-1}), or null (Markov)
+  float* P;              // [2][N][r] RNN head: Wh s_{i-1} of the group's rows, by step parity
+  __nv_bfloat16* shist;  // [K][N][r] RNN head: the state of every step (final-step bias)
   int32_t* draft;
   int32_t* out;
   int32_t* tau;
@@ -667,7 +670,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
     }
 
     // ---- Gather U[prev] rows (ctl->prev) into the B operand.
-    auto gather_u = [&](int nb_g) {
+    // B operand of step i: the Markov head's U[prev] rows, or the RNN head's
+    // state s_i = bf16(clamp(U[prev] + Wh s_{i-1}, -1, 1)) (Wh s_{i-1} from P,
+    // computed during the step before); at the final step (step == K) the RNN
+    // head takes each stopped row's saved state of its stop row instead.
+    auto gather_u = [&](int nb_g, int step) {
       const int cpr = a.r / 8;  // 16-byte chunks per row
       constexpr int kIt = N * 32 / kComputeThreads;  // r <= 256: at most 32 chunks per row
       uint4 val[kIt];
@@ -675,7 +682,43 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
       for (int t = 0; t < kIt; ++t) {  // all loads first, from clamped (valid) rows
         const int idx = tid + t * kComputeThreads;
         const int n = min(idx / cpr, N - 1), c = idx % cpr;
-        val[t] = __ldg(reinterpret_cast<const uint4*>(Ug + (size_t)ctl->prev[n] * a.r) + c);
+        if (a.Wh && step == K) {
+          const int j = ctl->alive[n] ? 0 : min(ctl->stoprow[n], K - 1);  // rows past the group: any saved row
+          val[t] = __ldcg(reinterpret_cast<const uint4*>(a.shist + ((size_t)j * N + n) * a.r) + c);
+        } else {
+          val[t] = __ldg(reinterpret_cast<const uint4*>(Ug + (size_t)ctl->prev[n] * a.r) + c);
+        }
+      }
+      if (a.Wh && step < K) {
+#pragma unroll
+        for (int t = 0; t < kIt; ++t) {
+          const int idx = tid + t * kComputeThreads;
+          const int n = min(idx / cpr, N - 1), c = idx % cpr;
+          float pw[8];
+          if (step > 0) {
+            const float4* pp = reinterpret_cast<const float4*>(a.P + ((size_t)(step & 1) * N + n) * a.r + c * 8);
+            const float4 p0 = __ldcg(pp), p1 = __ldcg(pp + 1);
+            pw[0] = p0.x; pw[1] = p0.y; pw[2] = p0.z; pw[3] = p0.w;
+            pw[4] = p1.x; pw[5] = p1.y; pw[6] = p1.z; pw[7] = p1.w;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) pw[e] = 0.f;
+          }
+          float x[8];
+          bf16x8(val[t], x);
+          uint32_t h[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float lo_ = fminf(fmaxf(__fadd_rn(x[2 * e], pw[2 * e]), -1.f), 1.f);
+            const float hi_ = fminf(fmaxf(__fadd_rn(x[2 * e + 1], pw[2 * e + 1]), -1.f), 1.f);
+            const __nv_bfloat162 bb = __floats2bfloat162_rn(lo_, hi_);
+            h[e] = *reinterpret_cast<const uint32_t*>(&bb);
+          }
+          val[t] = make_uint4(h[0], h[1], h[2], h[3]);
+          // the state of this step, for a final-step bias at this row
+          if (cta == 0 && idx < N * cpr && idx / cpr < nb_g)
+            *(reinterpret_cast<uint4*>(a.shist + ((size_t)step * N + idx / cpr) * a.r) + c) = val[t];
+        }
       }
 #pragma unroll
       for (int t = 0; t < kIt; ++t) {
@@ -799,8 +842,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
       }
       {  // warp w: rank rows [w*ks, w*ks + ks)
         const int ks = (a.r + 7) / 8, k0 = warp * ks, k1 = min(a.r, k0 + ks);
-        const int prev = ctl->prev[n];
-        const float uval = k0 + lane < k1 ? ld_elem(Ug, (int64_t)prev * a.r + k0 + lane) : 0.f;
+        // the bias operand of the row: U[prev] (Markov head) or the RNN state in sU
+        float uval = 0.f;
+        if (k0 + lane < k1) {
+          const int kk = k0 + lane, c = kk >> 3;
+          uval = a.Wh ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                            sU + (size_t)(c >> 3) * N * 128 + n * 128 + (((c & 7) ^ (n & 7)) << 4) +
+                            (kk & 7) * 2))
+                      : ld_elem(Ug, (int64_t)ctl->prev[n] * a.r + kk);
+        }
         float wv[32];
 #pragma unroll
         for (int t = 0; t < 32; ++t) wv[t] = k0 + t < k1 ? ld_elem(Wg, (int64_t)(k0 + t) * V + vc) : 0.f;
@@ -1126,10 +1176,30 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
           ctl->prev[n] = p;
         }
         named_sync();
-        gather_u(nb_g);
+        gather_u(nb_g, i);
         // the next step's base logits into L2 while this step runs
         if (tid < nb_g && i + 1 < K)
           prefetch_l2_bulk(base + ((jb0 + tid) * K + i + 1) * V + vslice_lo, slice_bytes);
+        if (a.Wh && i + 1 < K) {
+          // RNN head: this CTA's share of Wh s_i for the next step (fp32 fmaf in
+          // ascending k), visible to every CTA after this step's grid barrier
+          const int cpr = a.r / 8;
+          for (int o = cta * kComputeThreads + tid; o < nb_g * a.r; o += G * kComputeThreads) {
+            const int n = o / a.r, j = o % a.r;
+            const uint4* wr = reinterpret_cast<const uint4*>(a.Wh + (size_t)j * a.r);
+            float acc = 0.f;
+            for (int c = 0; c < cpr; ++c) {
+              const uint4 sw = *reinterpret_cast<const uint4*>(sU + (size_t)(c >> 3) * N * 128 + n * 128 +
+                                                              (((c & 7) ^ (n & 7)) << 4));
+              float xs[8], xw[8];
+              bf16x8(sw, xs);
+              bf16x8(__ldg(wr + c), xw);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) acc = fmaf(xs[e], xw[e], acc);
+            }
+            a.P[((size_t)((i + 1) & 1) * N + n) * a.r + j] = acc;
+          }
+        }
         mark(g, i, 1);
 
         // ---------------- epilogue: z = bias + base, exact bucket statistics
@@ -1225,7 +1295,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         // this CTA's target partials of row i (and row K) are out; the target
         // warps may take the next row
         if (tid == 0) {
-          const uint32_t J = (uint32_t)(g * K + i);
+          const uint32_t J = (uint32_t)(t * K + i);  // target jobs of all earlier jobs and steps
           if (!mbar_wait_bounded(&ctl->tdone, J & 1, a.spin, &hdr->abort)) {
             record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_BREADY, cta, 5000 + i);
             ctl->abort_local = 1;
@@ -1294,7 +1364,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
                                        ctl->alive[n] ? 0.f : 1.f / ctl->zS[n]);
         }
         named_sync();
-        gather_u(nb_g);
+        gather_u(nb_g, K);
         if (tid < nb_g) {  // the final rows of this CTA's slice into L2
           const int64_t b = jb0 + tid;
           const bool alive = ctl->alive[tid] != 0;
@@ -1475,6 +1545,8 @@ size_t tok_bytes(int K, int N) { return a256(sizeof(int32_t) * 2 * (size_t)K * N
 size_t rec_bytes(int K, int N) { return a256(sizeof(RecT) * 2 * (size_t)(K + 1) * N); }
 size_t rtag_bytes(int K, int N) { return a256(sizeof(uint64_t) * 2 * (size_t)(K + 1) * N); }
 size_t gbk_bytes(const CycleGeom& g) { return a256(sizeof(float2) * (size_t)g.G * g.nc * 4 * g.N); }
+size_t rnn_p_bytes(int N, int r) { return a256(sizeof(float) * 2 * (size_t)N * r); }
+size_t rnn_hist_bytes(int K, int N, int r) { return a256(sizeof(__nv_bfloat16) * (size_t)K * N * r); }
 
 }  // namespace
 
@@ -1507,9 +1579,10 @@ bool cycle_tc_geometry(int B, int K, int V, int r, int dtype, uint32_t flags, in
   return true;
 }
 
-size_t cycle_tc_ws_bytes(int K, const CycleGeom& g) {
+size_t cycle_tc_ws_bytes(int K, int r, const CycleGeom& g) {
   return cycle_trace_bytes(K) + dpart_bytes(K, g.N) + tpart_bytes(K, g.N) + tok_bytes(K, g.N) +
-         rec_bytes(K, g.N) + rtag_bytes(K, g.N) + gbk_bytes(g);
+         rec_bytes(K, g.N) + rtag_bytes(K, g.N) + gbk_bytes(g) + rnn_p_bytes(g.N, r) +
+         rnn_hist_bytes(K, g.N, r);
 }
 
 cudaError_t launch_cycle_tc(const CycleLaunch& L, const CycleGeom& g, WsHeader* hdr, uint8_t* body,
@@ -1525,6 +1598,7 @@ cudaError_t launch_cycle_tc(const CycleLaunch& L, const CycleGeom& g, WsHeader* 
   a.vlen = L.vlen;
   a.conf = L.conf;
   a.next_token = L.next_token;
+  a.Wh = reinterpret_cast<const __nv_bfloat16*>(L.Wh);
   a.draft = L.draft;
   a.out = L.out;
   a.tau = L.tau;
@@ -1544,6 +1618,10 @@ cudaError_t launch_cycle_tc(const CycleLaunch& L, const CycleGeom& g, WsHeader* 
   a.rtag = reinterpret_cast<uint64_t*>(body);
   body += rtag_bytes(L.K, g.N);
   a.gbk = reinterpret_cast<float2*>(body);
+  body += gbk_bytes(g);
+  a.P = reinterpret_cast<float*>(body);
+  body += rnn_p_bytes(g.N, L.r);
+  a.shist = reinterpret_cast<__nv_bfloat16*>(body);
   a.nbk = g.nc * 4;
   a.nts = g.N == 64 ? ring_slots_tc<64>(L.r, g.nc)
                     : (g.N == 32 ? ring_slots_tc<32>(L.r, g.nc) : ring_slots_tc<16>(L.r, g.nc));

@@ -87,6 +87,7 @@ struct CycleLaunch {
   float conf_thr;       // prefix survival threshold for conf
   int32_t* next_token;  // [B] last emitted token per row, carried between cycles, or null
   int ncyc;             // cycles per launch (0 or 1: one)
+  const void* Wh;       // [r][r] RNN head recurrence, or null (Markov head; tensor-core cycle only)
   int32_t* draft;
   int32_t* out;
   int32_t* tau;
@@ -108,7 +109,7 @@ cudaError_t launch_cycle(const CycleLaunch& L, const CycleGeom& g, WsHeader* hdr
 // bucket statistics.  Geometry returns false for other shapes.
 bool cycle_tc_geometry(int B, int K, int V, int r, int dtype, uint32_t flags, int num_sms,
                        CycleGeom* g, const char** why);
-size_t cycle_tc_ws_bytes(int K, const CycleGeom& g);
+size_t cycle_tc_ws_bytes(int K, int r, const CycleGeom& g);
 cudaError_t launch_cycle_tc(const CycleLaunch& L, const CycleGeom& g, WsHeader* hdr, uint8_t* body,
                             const CUtensorMap* tmW, cudaStream_t st);
 

@@ -213,6 +213,26 @@ spec_status spec_decode_loop(const spec_params *p, int32_t n_cycles, const void 
                              float *p_draft, float *q_draft, int32_t *next_token, void *workspace,
                              spec_stream_t stream);
 
+/* One cycle with the RNN sequential head in place of the Markov head
+ * (aigest.pl "DeepSeek prezentuje DSpark", section "Innowacje w tworzeniu
+ * tokenów": an optional RNN head tracks the whole block prefix).  The pages
+ * give no formula; the reading implemented is an Elman recurrence in the
+ * Markov head's factors:
+ *   s_{-1} = 0,  s_i = bf16(clamp(U[prev_i] + Wh s_{i-1}, -1, 1)),  bias_i = s_i . W,
+ * prev_i as for the Markov head.  (Wh s_{i-1})[j] is the fp32 fmaf chain over
+ * k = 0..r-1 of s_{i-1}[k] * Wh[j, k] starting from 0, U[prev_i, j] is added
+ * after it, and the result is clamped and rounded to bf16 (nearest, ties to
+ * even), so the state is the same bit for bit on any implementation that
+ * follows these steps.  Wh [r, r] bf16 (device), row j holding the weights of
+ * output j.  The recurrence of step i + 1 is computed during step i across
+ * the CTAs, so only its state update stays on the sequential path.  Otherwise
+ * as spec_cycle.  Tensor-core path only (bf16, rank a multiple of 64 up to
+ * 256); other shapes return SPEC_ERR_UNSUPPORTED. */
+spec_status spec_cycle_rnn(const spec_params *p, const void *base, const void *target,
+                           const void *U, const void *W, const void *Wh,
+                           const int32_t *last_token, int32_t *draft, int32_t *out, int32_t *tau,
+                           float *p_draft, float *q_draft, void *workspace, spec_stream_t stream);
+
 /* spec_cycle without a workspace argument, for callers that cannot allocate
  * device memory when they run a cycle (code whose allocations all belong to a
  * framework pool, a host thread that must not call cudaMalloc because it

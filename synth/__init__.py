@@ -107,6 +107,15 @@ def make_loop(w: Workload, n_cycles: int, B: int | None = None, seed: int | None
                 U=cyc[0]["U"], W=cyc[0]["W"], last_token=cyc[0]["last_token"], conf=conf)
 
 
+def rnn_weights(w: Workload, scale: float | None = None, seed: int | None = None):
+    """RNN head recurrence Wh [r, r] ~ N(0, scale^2) (default 1/sqrt(r)), in the
+    workload's dtype."""
+    g = torch.Generator().manual_seed((w.seed if seed is None else seed) + 31337)
+    sc = (1.0 / np.sqrt(w.r)) if scale is None else scale
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    return (_randn(g, (w.r, w.r)) * sc).to(tdt)
+
+
 def to_numpy_raw(t: torch.Tensor) -> np.ndarray:
     """Raw storage for the oracle: bf16 as uint16 bit patterns, f32 as float32."""
     t = t.contiguous()

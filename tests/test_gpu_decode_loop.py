@@ -172,3 +172,20 @@ def test_decode_loop_bad_verify_length_reported():
     vlen = np.array([[1, 2, 3, 4, 5], [1, 0, 2, 2, 2]], np.int32)
     st, _ = gpu_loop(w, d, 2, seed=1, use_conf=False, vlen=vlen)
     assert st == sd.SPEC_ERR_INVALID_ARG
+
+
+def test_decode_loop_odd_groups_odd_k():
+    """Three groups of rows and an odd K over two cycles: the per-job counters
+    of the target warps and the compute warps stay in step across cycles."""
+    w = synth.Workload("loopodd", B=150, K=5, V=6000, r=64, dtype="bf16", sigma=0.4, seed=68,
+                       uw_std=0.2)
+    C = 3
+    d = synth.make_loop(w, C)
+    for greedy in (False, True):
+        st, g = gpu_loop(w, d, C, greedy=greedy, seed=31, cyc=2, thr=0.3)
+        assert st == sd.SPEC_OK, sd.status_string(st)
+        o = orc_loop(w, d, C, greedy=greedy, seed=31, cyc=2, thr=0.3)
+        f, sync = compare_loop(g, o, w.K)
+        note_near(f"loop_odd{'_greedy' if greedy else ''}", 2, C * w.B, f)
+        check_chain(g, C, w.B)
+        assert sync.sum() >= w.B // 2

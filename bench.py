@@ -161,10 +161,10 @@ def measured_peak():
     return 6650.0, "fallback"
 
 
-def recorded_traffic(h):
+def recorded_traffic(h, name="k_cycle_tc_c3"):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current kernel source."""
-    p = os.path.join(ROOT, "profiles", "k_cycle_c3_ncu.json")
+    p = os.path.join(ROOT, "profiles", f"{name}_ncu.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
@@ -494,7 +494,8 @@ def run_ours(args, rank, world, local_rank):
             "hbm_gbs_full_stream": achieved,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak,
-                         "traffic": recorded_traffic(h) if (call == "cycle" and args.workload == WORKLOAD) else None,
+                         "traffic": (recorded_traffic(h, {"cycle": "k_cycle_tc_c3", "verify": "k_verify_ee_c3"}[call])
+                                     if (call in ("cycle", "verify") and args.workload == WORKLOAD) else None),
                          "peak_kind": peak_kind,
                          "bytes_per_launch": fb, "early_exit_bytes_per_launch": eb,
                          "early_exit_achieved": eb / (per_step_ms / 1e3) / 1e9,

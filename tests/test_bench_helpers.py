@@ -1,6 +1,8 @@
 """Host-side pieces of bench.py (CPU only): the roofline byte counts, the clock
 sampler's windowing and the peak / traffic lookups."""
 import json
+
+import pytest
 import os
 import sys
 
@@ -58,11 +60,12 @@ def test_measured_peak_reads_the_driver_file():
         assert kind == "fallback" and peak == 6650.0
 
 
-def test_recorded_traffic_only_for_the_profiled_source():
-    assert bench.recorded_traffic("not-the-profiled-source") is None
-    p = os.path.join(ROOT, "profiles", "k_cycle_c3_ncu.json")
+@pytest.mark.parametrize("name", ["k_cycle_tc_c3", "k_verify_ee_c3"])
+def test_recorded_traffic_only_for_the_profiled_source(name):
+    assert bench.recorded_traffic("not-the-profiled-source", name) is None
+    p = os.path.join(ROOT, "profiles", f"{name}_ncu.json")
     d = json.load(open(p))
-    assert bench.recorded_traffic(d["csrc_hash"]) == d["dram_bytes_per_launch"]
+    assert bench.recorded_traffic(d["csrc_hash"], name) == d["dram_bytes_per_launch"]
 
 
 def test_clock_sampler_short_region_takes_the_nearest_samples():

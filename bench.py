@@ -106,6 +106,9 @@ class ClockSampler:
                 text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            t_end = time.time() + 5.0  # the first sample before anything is timed
+            while not self.samples and time.time() < t_end and self.proc.poll() is None:
+                time.sleep(0.02)
         except OSError:
             self.proc = None
         return self

@@ -189,3 +189,23 @@ def test_decode_loop_odd_groups_odd_k():
         note_near(f"loop_odd{'_greedy' if greedy else ''}", 2, C * w.B, f)
         check_chain(g, C, w.B)
         assert sync.sum() >= w.B // 2
+
+
+def test_decode_loop_wait_limit_gives_timeout_and_context_survives():
+    w = CASES[0][1]
+    C = 2
+    d = synth.make_loop(w, C, seed=69)
+    dd = {k: v.cuda() for k, v in d.items()}
+    p = sd.Params(B=w.B, K=w.K, V=w.V, r=w.r, dtype=w.dtype, seed=1, spin_limit=1)
+    ws = sd.make_workspace(p)
+    o = sd.alloc_outputs(p, n_cycles=C)
+    nt = torch.empty(w.B, dtype=torch.int32, device="cuda")
+    sd.decode_loop(p, C, dd["base"], dd["target"], dd["U"], dd["W"], dd["last_token"], o["draft"],
+                   o["out"], o["tau"], o["p_draft"], o["q_draft"], nt, ws, conf=dd["conf"],
+                   conf_threshold=0.3)
+    assert sd.sync_status(ws) == sd.SPEC_ERR_TIMEOUT
+    sd.workspace_init(ws)
+    st, g = gpu_loop(w, d, C, seed=1, thr=0.3, dd=dd)
+    assert st == sd.SPEC_OK
+    o2 = orc_loop(w, d, C, seed=1, thr=0.3)
+    compare_loop(g, o2, w.K)

@@ -158,3 +158,23 @@ def test_verify_kb_all_k_equals_verify_block():
                        kb=np.full(w.B, w.K, np.int32))
     for k in ("out", "tau", "p_draft", "q_draft"):
         np.testing.assert_array_equal(a[k], b[k], err_msg=k)
+
+
+def test_verify_wait_limit_gives_timeout_and_context_survives():
+    """spin_limit = 1: the first wait of the one-launch verification gives up,
+    SPEC_ERR_TIMEOUT is recorded, the copies in flight are drained, and the
+    next call on the same workspace is correct."""
+    w = CASES[0][1]
+    target, dl, drafts = make_verify_inputs(w)
+    p = sd.Params(B=w.B, K=w.K, V=w.V, r=0, dtype="bf16", temperature=1.2, seed=3, cycle=5,
+                  spin_limit=1)
+    ws = sd.make_workspace(p)
+    outs = sd.alloc_outputs(p)
+    args = (target.cuda(), dl.cuda(), torch.from_numpy(drafts).cuda())
+    sd.verify_block(p, *args, outs["out"], outs["tau"], outs["p_draft"], outs["q_draft"], ws)
+    assert sd.sync_status(ws) == sd.SPEC_ERR_TIMEOUT
+    sd.workspace_init(ws)
+    st, gpu, o = run_both(w, target, dl, drafts, "bf16", 1.2, False, seed=3, cyc=5)
+    assert st == sd.SPEC_OK
+    early_exit_q(gpu, o)
+    compare_cycle(gpu, o, w.K)

@@ -470,6 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
           ok = false;
           break;
         }
+        if (a.trace && cta == 0 && t == 0 && tw == 0 && lane == 0)
+          a.trace[(size_t)j * kTracePhases + 4] = globaltimer_ns();  // target job taken
         // this lane's row n = 2 l + tw and its verify length K_b
         const int nl = 2 * lane + tw;
         const bool inrow = nl < nb_g && nl < N;
@@ -569,6 +571,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         __threadfence();  // the partials are visible device-wide before the job is reported
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->tdone);
+        if (a.trace && cta == 0 && t == 0 && tw == 0 && lane == 0)
+          a.trace[(size_t)j * kTracePhases + 31] = globaltimer_ns();  // target job published
       }
     }
     // nothing in flight at exit
@@ -1222,9 +1226,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
             uint4 cb[NV];
 #pragma unroll
             for (int u = 0; u < NV; ++u) cb[u] = nb[u];
+            if (cl + 1 < ncc) issue(cl + 1);  // next chunk's base logits in flight meanwhile
             float z[NCOL];
             acc_tile(z);
-            if (cl + 1 < ncc) issue(cl + 1);  // next chunk's base logits in flight meanwhile
             const int vv0 = (chunk0 + cl) * kCH + q4 * 32 + tg * NCOL;
             const bool full = rowok && vv0 + NCOL <= V;  // every token of this lane is valid
             float x[8];
@@ -1240,12 +1244,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
             float m = -INFINITY;
             int32_t mi = 0x7fffffff;
             if (a.greedy) {
+              // four interleaved arg-max chains (lowest index on ties), then combined
+              float mv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+              int32_t mx[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
 #pragma unroll
               for (int ee = 0; ee < NCOL; ++ee)
-                if (z[ee] > m) {
-                  m = z[ee];
-                  mi = vv0 + ee;
+                if (z[ee] > mv[ee & 3]) {
+                  mv[ee & 3] = z[ee];
+                  mx[ee & 3] = vv0 + ee;
                 }
+              m = mv[0];
+              mi = mx[0];
+#pragma unroll
+              for (int c4 = 1; c4 < 4; ++c4) amax_combine(m, mi, mv[c4], mx[c4]);
 #pragma unroll
               for (int o = 1; o < L; o <<= 1) {
                 const float m2 = __shfl_xor_sync(FULL, m, o);
@@ -1254,12 +1265,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
               }
               amax_combine(pm, pi, m, mi);
             } else {
+              // four interleaved chains for the max and for the sum (short dependencies)
+              float mv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-              for (int ee = 0; ee < NCOL; ++ee) m = fmaxf(m, z[ee]);
+              for (int ee = 0; ee < NCOL; ++ee) mv[ee & 3] = fmaxf(mv[ee & 3], z[ee]);
+              m = fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3]));
               float sum = 0.f;
               if (m > -INFINITY) {
+                float sv[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int ee = 0; ee < NCOL; ++ee) sum += fexp2((z[ee] - m) * k);
+                for (int ee = 0; ee < NCOL; ++ee) sv[ee & 3] += fexp2((z[ee] - m) * k);
+                sum = (sv[0] + sv[1]) + (sv[2] + sv[3]);
               }
 #pragma unroll
               for (int o = 1; o < L; o <<= 1) {

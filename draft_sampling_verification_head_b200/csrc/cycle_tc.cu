@@ -55,7 +55,8 @@ constexpr int kMmaWarp = 9;
 constexpr int kTargetWarp0 = 10;     // warps 10 and 11: target row statistics
 constexpr int kThreads = 384;
 constexpr int kTSMax = 16;           // row-slice slots per target warp, at most
-constexpr int kNS = 6;               // W ring stages
+template <int N>
+constexpr int kNSof = N >= 128 ? 4 : 6;  // W ring stages (fewer beside a 128-row operand)
 constexpr int kKS = 4;               // MMA K-steps (16 rank rows each) per stage
 constexpr int kWChunk = kCH * 16 * 2;         // 4 KB: one K-step of one chunk
 constexpr int kWStage = kKS * kWChunk;        // 16 KB: 64 rank rows of one chunk
@@ -121,7 +122,7 @@ static_assert(sizeof(RecT) == 64, "records are four 16-byte words");
 
 template <int N>
 struct CtlT {
-  uint64_t wfull[kNS], wempty[kNS], dfull[2], dfree[2];
+  uint64_t wfull[kNSof<N>], wempty[kNSof<N>], dfull[2], dfree[2];
   uint64_t bready, tready, mmadone;
   uint64_t tfull[2][kTSMax];  // target row slices landed (one ring per target warp)
   uint64_t tgo, tdone;     // target job may start / has published its partials
@@ -273,8 +274,11 @@ SPEC_DEV float ld_elem<__nv_bfloat16>(const __nv_bfloat16* p, int64_t i) {
 template <int N>
 __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant__ ArgsTC a) {
   constexpr int NCOL = N / 2;           // columns (batch rows) per compute warp
-  constexpr int L = 32 / NCOL;          // lanes per row after the transpose
-  constexpr int NV = NCOL / 8;          // 16-byte words per lane and logit row
+  constexpr int NS = NCOL > 32 ? NCOL / 32 : 1;  // column slabs a warp takes in turn
+  constexpr int SC = NCOL / NS;         // columns per slab (at most 32)
+  constexpr int L = 32 / SC;            // lanes per row after the transpose
+  constexpr int NV = SC / 8;            // 16-byte words per lane and logit row
+  constexpr int kNS = kNSof<N>;         // W ring stages
   using T = __nv_bfloat16;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -282,9 +286,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
   const int nkb = a.r / 64;             // 64-rank blocks = W ring stages per chunk
   uint8_t* sW = smem;                                       // kNS x 16 KB
   uint8_t* sU = sW + (size_t)kNS * kWStage;                 // nkb x N x 128 B
-  float* sT = reinterpret_cast<float*>(sU + (size_t)nkb * N * 128);  // 8 x 32 x NCOL floats
+  float* sT = reinterpret_cast<float*>(sU + (size_t)nkb * N * 128);  // 8 x 32 x SC floats
   const size_t rslot = (size_t)a.nc * kCH * sizeof(__nv_bfloat16);  // one row slice of the CTA
-  uint8_t* sR = reinterpret_cast<uint8_t*>(sT + 8 * 32 * NCOL);      // 2 x nts row slices
+  uint8_t* sR = reinterpret_cast<uint8_t*>(sT + 8 * 32 * SC);        // 2 x nts row slices
   const int kTS = a.nts;
   CtlT<N>* ctl = reinterpret_cast<CtlT<N>*>(sR + 2 * kTS * rslot);
 
@@ -472,101 +476,103 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         }
         if (a.trace && cta == 0 && t == 0 && tw == 0 && lane == 0)
           a.trace[(size_t)j * kTracePhases + 4] = globaltimer_ns();  // target job taken
-        // this lane's row n = 2 l + tw and its verify length K_b
-        const int nl = 2 * lane + tw;
-        const bool inrow = nl < nb_g && nl < N;
-        const int kbl = inrow ? row_verify_len(a, gb0 + nl) : 0;
-        const bool verifying =
-            inrow && j < kbl && (j == 0 || *reinterpret_cast<volatile int32_t*>(&ctl->alive[nl]) != 0);
-        if (verifying && j + 1 < kbl) {  // the next job's target rows of this row into L2
-          const int64_t bb = gb0 + nl;
-          prefetch_l2_bulk(target + (bb * (K + 1) + j + 1) * V + vlo, bytes);
-          if (j + 2 == kbl) prefetch_l2_bulk(target + (bb * (K + 1) + kbl) * V + vlo, bytes);
-        }
-        // rows still verifying at position j (a snapshot: a row that stops
-        // meanwhile only costs an unused slice); items: (row, target row j)
-        // and, at a row's last verified position, (row, target row K_b)
-        const uint32_t rows = __ballot_sync(FULL, verifying);
-        const uint32_t lastm = __ballot_sync(FULL, verifying && j == kbl - 1);
-        uint32_t imask = rows, cmask = rows;
-        int isub = 0, csub = 0;
-        auto next_item = [&](uint32_t& m, int& sub, int& n, int& trow) {
-          if (!m) return false;
-          const int l = __ffs(m) - 1;
-          n = 2 * l + tw;
-          trow = sub == 0 ? j : j + 1;
-          if (((lastm >> l) & 1u) && sub == 0) {
-            sub = 1;
-          } else {
-            sub = 0;
-            m &= m - 1;
+          // this lane's row n = 2 l + tw (+ 64 h) and its verify length K_b
+        for (int h = 0; h < (N + 63) / 64 && ok; ++h) {
+          const int nl = 2 * lane + tw + 64 * h;
+          const bool inrow = nl < nb_g && nl < N;
+          const int kbl = inrow ? row_verify_len(a, gb0 + nl) : 0;
+          const bool verifying =
+              inrow && j < kbl && (j == 0 || *reinterpret_cast<volatile int32_t*>(&ctl->alive[nl]) != 0);
+          if (verifying && j + 1 < kbl) {  // the next job's target rows of this row into L2
+            const int64_t bb = gb0 + nl;
+            prefetch_l2_bulk(target + (bb * (K + 1) + j + 1) * V + vlo, bytes);
+            if (j + 2 == kbl) prefetch_l2_bulk(target + (bb * (K + 1) + kbl) * V + vlo, bytes);
           }
-          return true;
-        };
-        auto issue = [&]() {  // lane 0: one copy into the slot freed last
-          int n, trow;
-          if (!next_item(imask, isub, n, trow)) return;
-          const uint32_t slot = tu % kTS;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&ctl->tfull[tw][slot], bytes);
-            bulk_load(ring + slot * rslot,
-                      target + ((gb0 + n) * (K + 1) + trow) * V + vlo, bytes,
-                      &ctl->tfull[tw][slot], pol);
-          }
-          ++tu;
-        };
-        while (tu - tcn < (uint32_t)kTS && imask) issue();
-        int n, trow;
-        while (next_item(cmask, csub, n, trow)) {
-          const uint32_t slot = tcn % kTS;
-          if (!mbar_wait_bounded(&ctl->tfull[tw][slot], (tcn / kTS) & 1, a.spin, &hdr->abort)) {
-            if (lane == 0) record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_FULL, cta, 4000 + j);
-            ok = false;
-            break;
-          }
-          const uint4* sl = reinterpret_cast<const uint4*>(ring + slot * rslot);
-          float x[8];
-          float m = -INFINITY, sm = 0.f;
-          int32_t mi = 0x7fffffff;
-          for (int p = lane; p < npieces; p += 32) {
-            bf16x8(sl[p], x);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              if (a.greedy) {
-                if (x[e] > m) {
-                  m = x[e];
-                  mi = vlo + 8 * p + e;
-                }
-              } else {
-                m = fmaxf(m, x[e]);
-              }
+          // rows still verifying at position j (a snapshot: a row that stops
+          // meanwhile only costs an unused slice); items: (row, target row j)
+          // and, at a row's last verified position, (row, target row K_b)
+          const uint32_t rows = __ballot_sync(FULL, verifying);
+          const uint32_t lastm = __ballot_sync(FULL, verifying && j == kbl - 1);
+          uint32_t imask = rows, cmask = rows;
+          int isub = 0, csub = 0;
+          auto next_item = [&](uint32_t& m, int& sub, int& n, int& trow) {
+            if (!m) return false;
+            const int l = __ffs(m) - 1;
+            n = 2 * l + tw + 64 * h;
+            trow = sub == 0 ? j : j + 1;
+            if (((lastm >> l) & 1u) && sub == 0) {
+              sub = 1;
+            } else {
+              sub = 0;
+              m &= m - 1;
             }
-          }
-          if (!a.greedy && m > -INFINITY) {
+            return true;
+          };
+          auto issue = [&]() {  // lane 0: one copy into the slot freed last
+            int n, trow;
+            if (!next_item(imask, isub, n, trow)) return;
+            const uint32_t slot = tu % kTS;
+            if (lane == 0) {
+              mbar_arrive_expect_tx(&ctl->tfull[tw][slot], bytes);
+              bulk_load(ring + slot * rslot,
+                        target + ((gb0 + n) * (K + 1) + trow) * V + vlo, bytes,
+                        &ctl->tfull[tw][slot], pol);
+            }
+            ++tu;
+          };
+          while (tu - tcn < (uint32_t)kTS && imask) issue();
+          int n, trow;
+          while (next_item(cmask, csub, n, trow)) {
+            const uint32_t slot = tcn % kTS;
+            if (!mbar_wait_bounded(&ctl->tfull[tw][slot], (tcn / kTS) & 1, a.spin, &hdr->abort)) {
+              if (lane == 0) record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_FULL, cta, 4000 + j);
+              ok = false;
+              break;
+            }
+            const uint4* sl = reinterpret_cast<const uint4*>(ring + slot * rslot);
+            float x[8];
+            float m = -INFINITY, sm = 0.f;
+            int32_t mi = 0x7fffffff;
             for (int p = lane; p < npieces; p += 32) {
               bf16x8(sl[p], x);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) sm += fexp2((x[e] - m) * k);
+  #pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                if (a.greedy) {
+                  if (x[e] > m) {
+                    m = x[e];
+                    mi = vlo + 8 * p + e;
+                  }
+                } else {
+                  m = fmaxf(m, x[e]);
+                }
+              }
             }
-          }
-          __syncwarp();
-          ++tcn;
-          issue();  // the slot is free: the next slice is in flight while this one reduces
-#pragma unroll
-          for (int off = 16; off >= 1; off >>= 1) {
-            const float m2 = __shfl_xor_sync(FULL, m, off);
-            if (a.greedy) {
-              const int32_t i2 = __shfl_xor_sync(FULL, mi, off);
-              amax_combine(m, mi, m2, i2);
-            } else {
-              const float s2 = __shfl_xor_sync(FULL, sm, off);
-              ms_combine(m, sm, m2, s2, k);
+            if (!a.greedy && m > -INFINITY) {
+              for (int p = lane; p < npieces; p += 32) {
+                bf16x8(sl[p], x);
+  #pragma unroll
+                for (int e = 0; e < 8; ++e) sm += fexp2((x[e] - m) * k);
+              }
             }
+            __syncwarp();
+            ++tcn;
+            issue();  // the slot is free: the next slice is in flight while this one reduces
+  #pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) {
+              const float m2 = __shfl_xor_sync(FULL, m, off);
+              if (a.greedy) {
+                const int32_t i2 = __shfl_xor_sync(FULL, mi, off);
+                amax_combine(m, mi, m2, i2);
+              } else {
+                const float s2 = __shfl_xor_sync(FULL, sm, off);
+                ms_combine(m, sm, m2, s2, k);
+              }
+            }
+            if (lane == 0)
+              a.tpart[(((int64_t)par * (K + 1) + trow) * N + n) * kMaxG + cta] =
+                  a.greedy ? make_float2(m, __int_as_float(mi)) : make_float2(m, sm);
           }
-          if (lane == 0)
-            a.tpart[(((int64_t)par * (K + 1) + trow) * N + n) * kMaxG + cta] =
-                a.greedy ? make_float2(m, __int_as_float(mi)) : make_float2(m, sm);
-        }
+        }  // halves
         if (!ok) break;
         __threadfence();  // the partials are visible device-wide before the job is reported
         __syncwarp();
@@ -588,8 +594,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
     const int q4 = warp & 3;               // tensor-memory lane quadrant (32 tokens of a chunk)
     const int n0 = (warp >> 2) * NCOL;     // first column (batch row) of this warp
     const int jj = lane / L, tg = lane % L;
-    const int nrow = n0 + jj;              // the batch row this lane holds after the transpose
-    float* tbuf = sT + warp * 32 * NCOL;
+    // the batch row this lane holds after the transpose of slab s
+    auto slab_row = [&](int s) { return n0 + s * SC + jj; };
+    float* tbuf = sT + warp * 32 * SC;
     uint32_t cc = 0, nbar = 0;
     const uint32_t ev0 = ld_volatile_u32(&hdr->events);  // record tags of this launch start here
     bool failed = false;
@@ -680,11 +687,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
     // head takes each stopped row's saved state of its stop row instead.
     auto gather_u = [&](int nb_g, int step) {
       const int cpr = a.r / 8;  // 16-byte chunks per row
-      constexpr int kIt = N * 32 / kComputeThreads;  // r <= 256: at most 32 chunks per row
+      constexpr int kItAll = N * 32 / kComputeThreads;  // r <= 256: at most 32 chunks per row
+      constexpr int kIt = kItAll < 8 ? kItAll : 8;      // words in flight per thread
+      for (int t0 = 0; t0 < kItAll; t0 += kIt) {
       uint4 val[kIt];
 #pragma unroll
       for (int t = 0; t < kIt; ++t) {  // all loads first, from clamped (valid) rows
-        const int idx = tid + t * kComputeThreads;
+        const int idx = tid + (t0 + t) * kComputeThreads;
         const int n = min(idx / cpr, N - 1), c = idx % cpr;
         if (a.Wh && step == K) {
           const int j = ctl->alive[n] ? 0 : min(ctl->stoprow[n], K - 1);  // rows past the group: any saved row
@@ -696,7 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
       if (a.Wh && step < K) {
 #pragma unroll
         for (int t = 0; t < kIt; ++t) {
-          const int idx = tid + t * kComputeThreads;
+          const int idx = tid + (t0 + t) * kComputeThreads;
           const int n = min(idx / cpr, N - 1), c = idx % cpr;
           float pw[8];
           if (step > 0) {
@@ -726,13 +735,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
       }
 #pragma unroll
       for (int t = 0; t < kIt; ++t) {
-        const int idx = tid + t * kComputeThreads;
+        const int idx = tid + (t0 + t) * kComputeThreads;
         const int n = idx / cpr, c = idx % cpr;
         if (idx >= N * cpr) continue;
         const int ka = c >> 3, j = c & 7;
         *reinterpret_cast<uint4*>(sU + (size_t)ka * N * 128 + n * 128 + ((j ^ (n & 7)) << 4)) =
             n < nb_g ? val[t] : make_uint4(0, 0, 0, 0);
       }
+      }  // batches
       fence_proxy_async_smem();
       named_sync();
       if (tid == 0) mbar_arrive(&ctl->bready);
@@ -740,20 +750,26 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
 
     // Accumulator tile of the next chunk for this thread (lane = token, NCOL
     // columns), handed back to the MMA once loaded; then transposed.
-    auto acc_tile = [&](float (&z)[NCOL]) {
+    // (Slab s of the warp's columns; the accumulator is waited for at slab 0
+    // and handed back after the last slab.)
+    auto acc_tile = [&](float (&z)[SC], int s) {
       const uint32_t b = cc & 1;
-      if (!mbar_wait_bounded(&ctl->dfull[b], (cc >> 1) & 1, a.spin, &hdr->abort))
-        soft_fail(SPEC_ERR_TIMEOUT, SITE_MBAR_MMA, cta, (int)cc);
-      tc_fence_after();
-      float d[NCOL];
-      tmem_ld_cols<NCOL>(taddr + ((uint32_t)(q4 * 32) << 16) + DB + b * (uint32_t)N + (uint32_t)n0, d);
-      tc_fence_before();
+      if (s == 0) {
+        if (!mbar_wait_bounded(&ctl->dfull[b], (cc >> 1) & 1, a.spin, &hdr->abort))
+          soft_fail(SPEC_ERR_TIMEOUT, SITE_MBAR_MMA, cta, (int)cc);
+        tc_fence_after();
+      }
+      float d[SC];
+      tmem_ld_cols<SC>(taddr + ((uint32_t)(q4 * 32) << 16) + DB + b * (uint32_t)N + (uint32_t)(n0 + s * SC), d);
+      if (s == NS - 1) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->dfree[b]);
+        ++cc;
+      }
+      transpose_in<SC>(tbuf, d, lane);
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl->dfree[b]);
-      ++cc;
-      transpose_in<NCOL>(tbuf, d, lane);
-      __syncwarp();
-      transpose_out<NCOL>(tbuf, z, lane);
+      transpose_out<SC>(tbuf, z, lane);
       __syncwarp();
     };
 
@@ -1117,10 +1133,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
     };
     // Quadrant partials of one quantity (lanes with tg == 0 hold the row's
     // value over this warp's tokens) into the CTA partial per row.
-    auto put_quadrant = [&](float (*qa)[N], float (*qb)[N], float x, float y) {
+    auto put_quadrant = [&](float (*qa)[N], float (*qb)[N], float x, float y, int row) {
       if (tg == 0) {
-        qa[q4][nrow] = x;
-        qb[q4][nrow] = y;
+        qa[q4][row] = x;
+        qb[q4][row] = y;
       }
     };
 
@@ -1208,90 +1224,107 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
 
         // ---------------- epilogue: z = bias + base, exact bucket statistics
         {
-          const bool rowok = nrow < nb_g;
-          const int64_t brow = jb0 + (rowok ? nrow : 0);
-          const T* bsrc = base + (brow * K + i) * V;
-          float pm = -INFINITY, ps = 0.f;  // stochastic: (max, sum); greedy: arg-max value
-          int32_t pi = 0x7fffffff;         // greedy: arg-max index
+          // per slab: stochastic (max, sum); greedy arg-max (value, index)
+          float pm[NS], ps[NS];
+          int32_t pi[NS];
+#pragma unroll
+          for (int sl = 0; sl < NS; ++sl) {
+            pm[sl] = -INFINITY;
+            ps[sl] = 0.f;
+            pi[sl] = 0x7fffffff;
+          }
           uint4 nb[NV];
-          auto issue = [&](int cl) {
-            const int vv0 = (chunk0 + cl) * kCH + q4 * 32 + tg * NCOL;
+          auto issue = [&](int cl, int sl) {  // base logits of chunk cl, slab sl, this lane's row
+            const int nr = slab_row(sl);
+            const bool ok = nr < nb_g;
+            const T* bsrc = base + ((jb0 + (ok ? nr : 0)) * K + i) * V;
+            const int vv0 = (chunk0 + cl) * kCH + q4 * 32 + tg * SC;
 #pragma unroll
             for (int u = 0; u < NV; ++u)
-              nb[u] = (rowok && vv0 + 8 * u < V) ? __ldcs(reinterpret_cast<const uint4*>(bsrc + vv0 + 8 * u))
-                                                 : make_uint4(0, 0, 0, 0);
+              nb[u] = (ok && vv0 + 8 * u < V) ? __ldcs(reinterpret_cast<const uint4*>(bsrc + vv0 + 8 * u))
+                                              : make_uint4(0, 0, 0, 0);
           };
-          issue(0);
+          issue(0, 0);
           for (int cl = 0; cl < ncc; ++cl) {
-            uint4 cb[NV];
 #pragma unroll
-            for (int u = 0; u < NV; ++u) cb[u] = nb[u];
-            if (cl + 1 < ncc) issue(cl + 1);  // next chunk's base logits in flight meanwhile
-            float z[NCOL];
-            acc_tile(z);
-            const int vv0 = (chunk0 + cl) * kCH + q4 * 32 + tg * NCOL;
-            const bool full = rowok && vv0 + NCOL <= V;  // every token of this lane is valid
-            float x[8];
+            for (int sl = 0; sl < NS; ++sl) {
+              const int nr = slab_row(sl);
+              const bool rowok = nr < nb_g;
+              uint4 cb[NV];
 #pragma unroll
-            for (int u = 0; u < NV; ++u) {
-              bf16x8(cb[u], x);
+              for (int u = 0; u < NV; ++u) cb[u] = nb[u];
+              // the next tile's base logits in flight meanwhile
+              if (sl + 1 < NS) issue(cl, sl + 1);
+              else if (cl + 1 < ncc) issue(cl + 1, 0);
+              float z[SC];
+              acc_tile(z, sl);
+              const int vv0 = (chunk0 + cl) * kCH + q4 * 32 + tg * SC;
+              const bool full = rowok && vv0 + SC <= V;  // every token of this lane is valid
+              float x[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const int ee = 8 * u + e;
-                z[ee] = (full || (rowok && vv0 + ee < V)) ? z[ee] + x[e] : -INFINITY;
-              }
-            }
-            float m = -INFINITY;
-            int32_t mi = 0x7fffffff;
-            if (a.greedy) {
-              // four interleaved arg-max chains (lowest index on ties), then combined
-              float mv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-              int32_t mx[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
+              for (int u = 0; u < NV; ++u) {
+                bf16x8(cb[u], x);
 #pragma unroll
-              for (int ee = 0; ee < NCOL; ++ee)
-                if (z[ee] > mv[ee & 3]) {
-                  mv[ee & 3] = z[ee];
-                  mx[ee & 3] = vv0 + ee;
+                for (int e = 0; e < 8; ++e) {
+                  const int ee = 8 * u + e;
+                  z[ee] = (full || (rowok && vv0 + ee < V)) ? z[ee] + x[e] : -INFINITY;
                 }
-              m = mv[0];
-              mi = mx[0];
-#pragma unroll
-              for (int c4 = 1; c4 < 4; ++c4) amax_combine(m, mi, mv[c4], mx[c4]);
-#pragma unroll
-              for (int o = 1; o < L; o <<= 1) {
-                const float m2 = __shfl_xor_sync(FULL, m, o);
-                const int32_t i2 = __shfl_xor_sync(FULL, mi, o);
-                amax_combine(m, mi, m2, i2);
               }
-              amax_combine(pm, pi, m, mi);
-            } else {
-              // four interleaved chains for the max and for the sum (short dependencies)
-              float mv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+              float m = -INFINITY;
+              int32_t mi = 0x7fffffff;
+              if (a.greedy) {
+                // four interleaved arg-max chains (lowest index on ties), then combined
+                float mv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                int32_t mx[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
 #pragma unroll
-              for (int ee = 0; ee < NCOL; ++ee) mv[ee & 3] = fmaxf(mv[ee & 3], z[ee]);
-              m = fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3]));
-              float sum = 0.f;
-              if (m > -INFINITY) {
-                float sv[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int ee = 0; ee < SC; ++ee)
+                  if (z[ee] > mv[ee & 3]) {
+                    mv[ee & 3] = z[ee];
+                    mx[ee & 3] = vv0 + ee;
+                  }
+                m = mv[0];
+                mi = mx[0];
 #pragma unroll
-                for (int ee = 0; ee < NCOL; ++ee) sv[ee & 3] += fexp2((z[ee] - m) * k);
-                sum = (sv[0] + sv[1]) + (sv[2] + sv[3]);
+                for (int c4 = 1; c4 < 4; ++c4) amax_combine(m, mi, mv[c4], mx[c4]);
+#pragma unroll
+                for (int o = 1; o < L; o <<= 1) {
+                  const float m2 = __shfl_xor_sync(FULL, m, o);
+                  const int32_t i2 = __shfl_xor_sync(FULL, mi, o);
+                  amax_combine(m, mi, m2, i2);
+                }
+                amax_combine(pm[sl], pi[sl], m, mi);
+              } else {
+                // four interleaved chains for the max and for the sum (short dependencies)
+                float mv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int ee = 0; ee < SC; ++ee) mv[ee & 3] = fmaxf(mv[ee & 3], z[ee]);
+                m = fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3]));
+                float sum = 0.f;
+                if (m > -INFINITY) {
+                  float sv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                  for (int ee = 0; ee < SC; ++ee) sv[ee & 3] += fexp2((z[ee] - m) * k);
+                  sum = (sv[0] + sv[1]) + (sv[2] + sv[3]);
+                }
+#pragma unroll
+                for (int o = 1; o < L; o <<= 1) {
+                  const float m2 = __shfl_xor_sync(FULL, m, o), s2 = __shfl_xor_sync(FULL, sum, o);
+                  ms_combine(m, sum, m2, s2, k);
+                }
+                if (tg == 0 && rowok)
+                  a.gbk[((size_t)cta * a.nbk + cl * 4 + q4) * N + nr] = make_float2(m, sum);
+                ms_combine(pm[sl], ps[sl], m, sum, k);
               }
-#pragma unroll
-              for (int o = 1; o < L; o <<= 1) {
-                const float m2 = __shfl_xor_sync(FULL, m, o), s2 = __shfl_xor_sync(FULL, sum, o);
-                ms_combine(m, sum, m2, s2, k);
-              }
-              if (tg == 0 && rowok)
-                a.gbk[((size_t)cta * a.nbk + cl * 4 + q4) * N + nrow] = make_float2(m, sum);
-              ms_combine(pm, ps, m, sum, k);
             }
             if (trace && g == 0 && cl < 8) trace[(size_t)i * kTracePhases + 16 + cl] = globaltimer_ns();
           }
-          if (a.greedy)
-            put_quadrant(ctl->qa, ctl->qb, pm, __int_as_float(pi));
-          else
-            put_quadrant(ctl->qa, ctl->qb, pm, ps);
+#pragma unroll
+          for (int sl = 0; sl < NS; ++sl) {
+            if (a.greedy)
+              put_quadrant(ctl->qa, ctl->qb, pm[sl], __int_as_float(pi[sl]), slab_row(sl));
+            else
+              put_quadrant(ctl->qa, ctl->qb, pm[sl], ps[sl], slab_row(sl));
+          }
         }
         named_sync();
         mark(g, i, 2);
@@ -1390,17 +1423,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         }
         mark(g, K, 1);
         {
-          const bool rowok = nrow < nb_g;
-          const bool ralive = rowok && ctl->alive[nrow] != 0;
-          const int frow = ralive ? ctl->kb[nrow] : (rowok ? ctl->stoprow[nrow] : 0);
-          const int64_t brow = jb0 + (rowok ? nrow : 0);
-          const T* tsrc = target + (brow * (K + 1) + frow) * V;
-          const T* bsrc = base + (brow * K + min(frow, K - 1)) * V;
-          const float4 c = rowok ? ctl->fcst[nrow] : make_float4(0.f, 0.f, 0.f, 0.f);
-          float R = 0.f, P = 0.f;
+          float Rs[NS], Ps[NS];
+#pragma unroll
+          for (int sl = 0; sl < NS; ++sl) Rs[sl] = Ps[sl] = 0.f;
           uint4 nt[NV], nb[NV];
-          auto issue = [&](int cl) {
-            const int vv0 = (chunk0 + cl) * kCH + q4 * 32 + tg * NCOL;
+          // the stop row's (or bonus row's) target logits and, for stopped rows,
+          // the draft base of that row: chunk cl, slab sl, this lane's row
+          auto issue = [&](int cl, int sl) {
+            const int nr = slab_row(sl);
+            const bool rowok = nr < nb_g;
+            const bool ralive = rowok && ctl->alive[nr] != 0;
+            const int frow = ralive ? ctl->kb[nr] : (rowok ? ctl->stoprow[nr] : 0);
+            const int64_t brow = jb0 + (rowok ? nr : 0);
+            const T* tsrc = target + (brow * (K + 1) + frow) * V;
+            const T* bsrc = base + (brow * K + min(frow, K - 1)) * V;
+            const int vv0 = (chunk0 + cl) * kCH + q4 * 32 + tg * SC;
 #pragma unroll
             for (int u = 0; u < NV; ++u) {
               const int vv = vv0 + 8 * u;
@@ -1410,48 +1447,56 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
                                       : make_uint4(0, 0, 0, 0);
             }
           };
-          issue(0);
+          issue(0, 0);
           for (int cl = 0; cl < ncc; ++cl) {
-            uint4 ct[NV], cb[NV];
 #pragma unroll
-            for (int u = 0; u < NV; ++u) {
-              ct[u] = nt[u];
-              cb[u] = nb[u];
-            }
-            float z[NCOL];
-            acc_tile(z);  // the bias at the stop row (alive rows: unused)
-            if (cl + 1 < ncc) issue(cl + 1);  // next chunk's logits in flight meanwhile
-            const int vv0 = (chunk0 + cl) * kCH + q4 * 32 + tg * NCOL;
-            const bool any = rowok && vv0 < V;
-            float r = 0.f, p = 0.f;
-            float xt[8], xb[8];
+            for (int sl = 0; sl < NS; ++sl) {
+              const int nr = slab_row(sl);
+              const bool rowok = nr < nb_g;
+              const float4 c = rowok ? ctl->fcst[nr] : make_float4(0.f, 0.f, 0.f, 0.f);
+              uint4 ct[NV], cb[NV];
 #pragma unroll
-            for (int u = 0; u < NV; ++u) {
-              bf16x8(ct[u], xt);
-              bf16x8(cb[u], xb);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const bool ok = any && vv0 + 8 * u + e < V;
-                // residual mass and target mass; a row that accepted every
-                // draft has 1 / draft sum = 0: r = p
-                const float pe = fexp2((xt[e] - c.x) * k) * c.y;
-                const float qe = c.w != 0.f ? fexp2((z[8 * u + e] + xb[e] - c.z) * k) * c.w : 0.f;
-                r += ok ? fmaxf(pe - qe, 0.f) : 0.f;
-                p += ok ? pe : 0.f;
+              for (int u = 0; u < NV; ++u) {
+                ct[u] = nt[u];
+                cb[u] = nb[u];
               }
-            }
+              if (sl + 1 < NS) issue(cl, sl + 1);  // the next tile's logits in flight meanwhile
+              else if (cl + 1 < ncc) issue(cl + 1, 0);
+              float z[SC];
+              acc_tile(z, sl);  // the bias at the stop row (alive rows: unused)
+              const int vv0 = (chunk0 + cl) * kCH + q4 * 32 + tg * SC;
+              const bool any = rowok && vv0 < V;
+              float r = 0.f, p = 0.f;
+              float xt[8], xb[8];
 #pragma unroll
-            for (int o = 1; o < L; o <<= 1) {
-              r += __shfl_xor_sync(FULL, r, o);
-              p += __shfl_xor_sync(FULL, p, o);
+              for (int u = 0; u < NV; ++u) {
+                bf16x8(ct[u], xt);
+                bf16x8(cb[u], xb);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  const bool ok = any && vv0 + 8 * u + e < V;
+                  // residual mass and target mass; a row that accepted every
+                  // draft has 1 / draft sum = 0: r = p
+                  const float pe = fexp2((xt[e] - c.x) * k) * c.y;
+                  const float qe = c.w != 0.f ? fexp2((z[8 * u + e] + xb[e] - c.z) * k) * c.w : 0.f;
+                  r += ok ? fmaxf(pe - qe, 0.f) : 0.f;
+                  p += ok ? pe : 0.f;
+                }
+              }
+#pragma unroll
+              for (int o = 1; o < L; o <<= 1) {
+                r += __shfl_xor_sync(FULL, r, o);
+                p += __shfl_xor_sync(FULL, p, o);
+              }
+              if (tg == 0 && rowok)
+                a.gbk[((size_t)cta * a.nbk + cl * 4 + q4) * N + nr] = make_float2(r, p);
+              Rs[sl] += r;
+              Ps[sl] += p;
             }
-            if (tg == 0 && rowok)
-              a.gbk[((size_t)cta * a.nbk + cl * 4 + q4) * N + nrow] = make_float2(r, p);
-            R += r;
-            P += p;
             if (trace && g == 0 && cl < 8) trace[(size_t)K * kTracePhases + 16 + cl] = globaltimer_ns();
           }
-          put_quadrant(ctl->qa, ctl->qb, R, P);
+#pragma unroll
+          for (int sl = 0; sl < NS; ++sl) put_quadrant(ctl->qa, ctl->qb, Rs[sl], Ps[sl], slab_row(sl));
         }
         named_sync();
         mark(g, K, 2);
@@ -1525,10 +1570,11 @@ constexpr size_t kSmemBudget = 227 * 1024;
 template <int N>
 size_t smem_fixed_tc(int r) {
   constexpr int NCOL = N / 2;
+  constexpr int SC = NCOL > 32 ? 32 : NCOL;
   size_t s = 1024;  // alignment slack
-  s += (size_t)kNS * kWStage;
+  s += (size_t)kNSof<N> * kWStage;
   s += (size_t)(r / 64) * N * 128;
-  s += (size_t)8 * 32 * NCOL * sizeof(float);
+  s += (size_t)8 * 32 * SC * sizeof(float);
   s += sizeof(CtlT<N>);
   return s;
 }
@@ -1581,11 +1627,13 @@ bool cycle_tc_geometry(int B, int K, int V, int r, int dtype, uint32_t flags, in
     *why = "more CTAs than the kernel's partial buffers allow";
     return false;
   }
-  g->N = B > 32 ? 64 : (B > 16 ? 32 : 16);
+  g->N = B > 64 ? 128 : (B > 32 ? 64 : (B > 16 ? 32 : 16));
   g->tc = true;
-  g->smem = g->N == 64 ? smem_bytes_tc<64>(r, nc)
+  g->smem = g->N == 128 ? smem_bytes_tc<128>(r, nc)
+          : g->N == 64 ? smem_bytes_tc<64>(r, nc)
                         : (g->N == 32 ? smem_bytes_tc<32>(r, nc) : smem_bytes_tc<16>(r, nc));
-  const int nts = g->N == 64 ? ring_slots_tc<64>(r, nc)
+  const int nts = g->N == 128 ? ring_slots_tc<128>(r, nc)
+                : g->N == 64 ? ring_slots_tc<64>(r, nc)
                              : (g->N == 32 ? ring_slots_tc<32>(r, nc) : ring_slots_tc<16>(r, nc));
   if (nts < 2 || g->smem > kSmemBudget) {
     *why = "shared memory budget exceeded";
@@ -1639,7 +1687,8 @@ cudaError_t launch_cycle_tc(const CycleLaunch& L, const CycleGeom& g, WsHeader* 
   body += rnn_p_bytes(g.N, L.r);
   a.shist = reinterpret_cast<__nv_bfloat16*>(body);
   a.nbk = g.nc * 4;
-  a.nts = g.N == 64 ? ring_slots_tc<64>(L.r, g.nc)
+  a.nts = g.N == 128 ? ring_slots_tc<128>(L.r, g.nc)
+        : g.N == 64 ? ring_slots_tc<64>(L.r, g.nc)
                     : (g.N == 32 ? ring_slots_tc<32>(L.r, g.nc) : ring_slots_tc<16>(L.r, g.nc));
   a.B = L.B;
   a.K = L.K;
@@ -1650,7 +1699,7 @@ cudaError_t launch_cycle_tc(const CycleLaunch& L, const CycleGeom& g, WsHeader* 
   a.nchunks = g.nchunks;
   a.greedy = L.greedy;
   a.ngroups = (L.B + g.N - 1) / g.N;
-  a.NT = std::min(kMaxNT, g.nc);
+  a.NT = std::min(std::min(kMaxNT, g.nc), (512 - 2 * g.N) / 128);  // TMEM: accumulators first
   a.k = L.greedy ? 1.0f : 1.4426950408889634f / L.temperature;
   a.conf_thr = L.conf_thr;
   a.ncyc = std::max(L.ncyc, 1);
@@ -1661,7 +1710,8 @@ cudaError_t launch_cycle_tc(const CycleLaunch& L, const CycleGeom& g, WsHeader* 
   switch (g.N) {
     case 16: return launch_tc<16>(a, g.G, g.smem, st);
     case 32: return launch_tc<32>(a, g.G, g.smem, st);
-    default: return launch_tc<64>(a, g.G, g.smem, st);
+    case 64: return launch_tc<64>(a, g.G, g.smem, st);
+    default: return launch_tc<128>(a, g.G, g.smem, st);
   }
 }
 

@@ -212,10 +212,15 @@ CASES = [
                                          sigma=0.4, seed=68, uw_std=0.1), True, 0.9),
     ("n64_full_greedy", synth.Workload("n64f", B=64, K=8, V=32000, r=256, dtype="bf16",
                                        sigma=0.5, seed=69, uw_std=0.1), True, 1.0),
-    ("n64_two_groups", synth.Workload("n64g", B=100, K=4, V=9000, r=64, dtype="bf16",
+    ("n128_one_group", synth.Workload("n64g", B=100, K=4, V=9000, r=64, dtype="bf16",
                                       sigma=0.6, seed=70, uw_std=0.3), False, 1.0),
-    ("n64_two_groups_greedy", synth.Workload("n64g", B=100, K=4, V=9000, r=64, dtype="bf16",
+    ("n128_one_group_greedy", synth.Workload("n64g", B=100, K=4, V=9000, r=64, dtype="bf16",
                                              sigma=0.6, seed=70, uw_std=0.3), True, 1.0),
+    # 128-row groups: 200 rows are a full group and a ragged one, run in turn
+    ("n128_two_groups", synth.Workload("n128g", B=200, K=5, V=9000, r=128, dtype="bf16",
+                                       sigma=0.5, seed=75, uw_std=0.3), False, 0.9),
+    ("n128_two_groups_greedy", synth.Workload("n128g", B=200, K=5, V=9000, r=128, dtype="bf16",
+                                              sigma=0.5, seed=75, uw_std=0.3), True, 0.9),
 ]
 
 

@@ -52,7 +52,8 @@ CASES = [
     ("two_groups", synth.Workload("rng", B=100, K=5, V=9000, r=128, dtype="bf16", sigma=0.3,
                                   seed=102, uw_std=0.2), 0.9),
     ("n16_rank256", synth.Workload("rn16", B=12, K=4, V=20000, r=256, dtype="bf16", sigma=0.6,
-                                   seed=103, uw_std=0.08), 1.0),
+                                   seed=103, uw_std=0.08), 1.0),    ("two_groups_n128", synth.Workload("rng2", B=160, K=4, V=7000, r=128, dtype="bf16",
+                                       sigma=0.4, seed=104, uw_std=0.2), 1.0),
 ]
 
 

@@ -68,7 +68,8 @@ CASES = [
     ("small", synth.Workload("kb", B=5, K=6, V=1000, r=64, dtype="bf16", sigma=0.4, seed=91,
                              uw_std=0.3), 1.0),
     ("two_groups", synth.Workload("kbg", B=100, K=5, V=9000, r=128, dtype="bf16", sigma=0.3,
-                                  seed=92, uw_std=0.2), 0.9),
+                                  seed=92, uw_std=0.2), 0.9),    ("two_groups_n128", synth.Workload("kbg2", B=190, K=5, V=9000, r=128, dtype="bf16",
+                                       sigma=0.3, seed=94, uw_std=0.2), 0.9),
 ]
 
 

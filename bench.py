@@ -43,10 +43,13 @@ def _strip_comments(src: str) -> str:
 
 
 def csrc_hash(root: str = ROOT) -> str:
-    """Fingerprint of the kernel sources, comments excluded: a recorded ncu
-    traffic figure stays valid while the code it measured is unchanged."""
+    """Fingerprint of the CUDA sources (.cu, .cuh), comments excluded: a
+    recorded ncu traffic figure stays valid while the code it measured is
+    unchanged.  Host-only C++ (.cpp) launches nothing and is left out."""
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(root, "draft_sampling_verification_head_b200", "csrc", "*"))):
+    csrc = os.path.join(root, "draft_sampling_verification_head_b200", "csrc")
+    files = glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))
+    for f in sorted(files):
         h.update(os.path.basename(f).encode())
         h.update(_strip_comments(open(f, encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]

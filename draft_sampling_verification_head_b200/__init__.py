@@ -37,6 +37,8 @@ _SIGS = {
     "spec_sync_status": (ctypes.c_int, [_P, _P]),
     "spec_cycle_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "spec_l2_persist": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
+    "spec_schedule_verify_len": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, _P,
+                                                 ctypes.c_int32, _P, _P]),
     "spec_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "spec_last_launch_count": (ctypes.c_int32, []),
     "spec_debug_philox": (ctypes.c_int, [_P, _P, _P, ctypes.c_int32, _P]),
@@ -229,6 +231,23 @@ def l2_persist(t, nbytes=None, stream=None):
     ptr = None if t is None else ctypes.c_void_p(t.data_ptr())
     n = 0 if t is None else (t.numel() * t.element_size() if nbytes is None else nbytes)
     _check(lib().spec_l2_persist(ptr, n, _stream(stream)), "spec_l2_persist")
+
+
+def schedule_verify_len(conf, sps):
+    """Verify length per request from confidence scores conf [B, K] and the
+    steps-per-second table sps [n] (host arrays).  Returns (verify_len [B]
+    int32, expected tokens per step, expected tokens per second)."""
+    import numpy as np
+    c = np.ascontiguousarray(conf, dtype=np.float32)
+    s = np.ascontiguousarray(sps, dtype=np.float64)
+    if c.ndim != 2 or s.ndim != 1:
+        raise ValueError("conf must be [B, K] and sps one-dimensional")
+    kb = np.empty(c.shape[0], np.int32)
+    ex = np.zeros(2, np.float64)
+    _check(lib().spec_schedule_verify_len(c.ctypes.data, c.shape[0], c.shape[1], s.ctypes.data,
+                                          s.shape[0], kb.ctypes.data, ex.ctypes.data),
+           "spec_schedule_verify_len")
+    return kb, float(ex[0]), float(ex[1])
 
 
 def last_launch_count() -> int:

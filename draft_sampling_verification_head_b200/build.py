@@ -11,7 +11,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libspecdec.so")
 SOURCES = ["api.cu", "bias_gemm.cu", "verify.cu", "verify_ee.cu", "cycle.cu", "cycle_tc.cu",
-           "noalloc.cu"]
+           "noalloc.cu", "schedule.cpp"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "--threads", "4", "-Xptxas", "-v"]
 

@@ -252,6 +252,31 @@ spec_status spec_cycle_noalloc(const spec_params *p, const void *base, const voi
                                int32_t *draft, int32_t *out, int32_t *tau, float *p_draft,
                                float *q_draft, int32_t *status_out, spec_stream_t stream);
 
+/* Verify-length scheduler (host logic; no device work, no stream, callable
+ * without a GPU).  mkdocs.reaper.mx DeepSeek-V4.1-Flash "06-extensions", DSpark
+ * table: the scheduler chooses each request's verify length from the prefix
+ * survival probabilities of the confidence head and the engine's throughput
+ * curve measured beforehand, to maximise expected throughput under the current
+ * load; aigest.pl "DeepSeek prezentuje DSpark", "Optymalizacja weryfikacji i
+ * wydajności": that curve is SPS(B), profiled once at start-up.  Reading: with
+ * S_{b,i} = prod_{j<=i} clamp(conf[b][j], 0, 1) (a NaN score counts as 0),
+ * choose k_b in 1..K maximising
+ *   E * SPS(M),  E = sum_b (1 + sum_{i<k_b} S_{b,i}),  M = sum_b (k_b + 1)
+ * (expected tokens per step times steps per second for a target pass over M
+ * rows); among equal maxima the smallest total length, among allocations of
+ * that total the one taking the larger S first, ties to the lower row b.
+ *   conf        [B, K] float, host    confidence scores per draft position
+ *   sps         [n_sps] double, host  steps per second of a target pass over m
+ *                                     rows, m = 0 .. n_sps-1; 0 past the table
+ *   verify_len  [B] int32, host       output k_b, ready for spec_cycle_kb
+ *   expected    [2] double, host      output (E, E * SPS(M)); may be NULL
+ * Errors: SPEC_ERR_INVALID_ARG for a NULL pointer, B or K < 1, B*K > 2^26,
+ * n_sps < 1, or an SPS entry that is negative, NaN or infinite (nothing is
+ * written then).  Cost O(BK log BK) on the calling thread. */
+spec_status spec_schedule_verify_len(const float *conf, int32_t B, int32_t K,
+                                     const double *sps, int32_t n_sps, int32_t *verify_len,
+                                     double *expected);
+
 /* Keep [ptr, ptr + bytes) resident in L2 for kernels later launched on
  * `stream` (a persisting access-policy window on the stream; the persisting
  * L2 carve-out of the calling process's context is raised to fit, up to the

@@ -530,28 +530,43 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
               break;
             }
             const uint4* sl = reinterpret_cast<const uint4*>(ring + slot * rslot);
-            float x[8];
             float m = -INFINITY, sm = 0.f;
             int32_t mi = 0x7fffffff;
-            for (int p = lane; p < npieces; p += 32) {
-              bf16x8(sl[p], x);
+            // one pass: the lane's pieces p = lane + 32 u are read four at a
+            // time (their shared-memory latencies overlap); stochastic rows
+            // keep a running (max, sum) rescaled once per piece
+            for (int p0 = lane; p0 < npieces; p0 += 128) {
+              uint4 w4[4];
   #pragma unroll
-              for (int e = 0; e < 8; ++e) {
+              for (int u = 0; u < 4; ++u)
+                w4[u] = p0 + 32 * u < npieces ? sl[p0 + 32 * u] : make_uint4(0, 0, 0, 0);
+  #pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const int p = p0 + 32 * u;
+                if (p >= npieces) break;
+                float x[8];
+                bf16x8(w4[u], x);
                 if (a.greedy) {
-                  if (x[e] > m) {
-                    m = x[e];
-                    mi = vlo + 8 * p + e;
-                  }
-                } else {
-                  m = fmaxf(m, x[e]);
-                }
-              }
-            }
-            if (!a.greedy && m > -INFINITY) {
-              for (int p = lane; p < npieces; p += 32) {
-                bf16x8(sl[p], x);
   #pragma unroll
-                for (int e = 0; e < 8; ++e) sm += fexp2((x[e] - m) * k);
+                  for (int e = 0; e < 8; ++e)
+                    if (x[e] > m) {
+                      m = x[e];
+                      mi = vlo + 8 * p + e;
+                    }
+                } else {
+                  const float m8 = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])),
+                                         fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
+                  const float mn = fmaxf(m, m8);
+                  if (mn > -INFINITY) {
+                    float sv[4];
+  #pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                      sv[e] = fexp2((x[e] - mn) * k) + fexp2((x[e + 4] - mn) * k);
+                    const float s8 = (sv[0] + sv[1]) + (sv[2] + sv[3]);
+                    sm = m > -INFINITY ? fmaf(sm, fexp2((m - mn) * k), s8) : s8;
+                    m = mn;
+                  }
+                }
               }
             }
             __syncwarp();
@@ -871,13 +886,38 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
                             (kk & 7) * 2))
                       : ld_elem(Ug, (int64_t)ctl->prev[n] * a.r + kk);
         }
-        float wv[32];
+        // lane l: the 8 tokens v0 + 8 (l & 3) .. + 7 of rank rows k0 + (l >> 2) + 8 j,
+        // one 16-byte load per rank row (V % 8 == 0: a group of 8 is all in or all out)
+        const int g8 = lane & 3, rs = lane >> 2;
+        const int vg = v0 + 8 * g8;
+        uint4 wq[4];
 #pragma unroll
-        for (int t = 0; t < 32; ++t) wv[t] = k0 + t < k1 ? ld_elem(Wg, (int64_t)(k0 + t) * V + vc) : 0.f;
-        float part = 0.f;
+        for (int j = 0; j < 4; ++j) {
+          const int kk = k0 + rs + 8 * j;
+          wq[j] = (vg < V && kk < k1)
+                      ? __ldg(reinterpret_cast<const uint4*>(Wg + (int64_t)kk * V + vg))
+                      : make_uint4(0, 0, 0, 0);
+        }
+        float acc8[8];
 #pragma unroll
-        for (int t = 0; t < 32; ++t) part = fmaf(__shfl_sync(FULL, uval, t), wv[t], part);
-        ctl->zpart[warp][lane] = part;
+        for (int e = 0; e < 8; ++e) acc8[e] = 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float u = __shfl_sync(FULL, uval, rs + 8 * j);
+          float xw[8];
+          bf16x8(wq[j], xw);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc8[e] = fmaf(u, xw[e], acc8[e]);
+        }
+        // the 8 lanes of a token group (equal l & 3) hold its rank rows
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc8[e] += __shfl_xor_sync(FULL, acc8[e], off);
+        if (rs == 0) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ctl->zpart[warp][8 * g8 + e] = acc8[e];
+        }
       }
       named_sync();
       if (j == 0 && kind == 0) mark(g, i, 15);

@@ -42,17 +42,31 @@ def _strip_comments(src: str) -> str:
     return "\n".join(l.rstrip() for l in src.splitlines() if l.strip())
 
 
-def csrc_hash(root: str = ROOT) -> str:
-    """Fingerprint of the CUDA sources (.cu, .cuh), comments excluded: a
-    recorded ncu traffic figure stays valid while the code it measured is
-    unchanged.  Host-only C++ (.cpp) launches nothing and is left out."""
+# the sources each profiled kernel is built from (besides the shared headers)
+PROFILED_SOURCES = {"k_cycle_tc_c3": ("cycle_tc.cu",), "k_verify_ee_c3": ("verify_ee.cu",)}
+SHARED_HEADERS = ("common.cuh", "kernels.cuh")
+
+
+def csrc_hash(files=None, root: str = ROOT) -> str:
+    """Fingerprint of CUDA sources, comments excluded: the given kernel files
+    and the shared headers, or every .cu / .cuh file.  A recorded ncu traffic
+    figure stays valid while the code it measured is unchanged.  Host-only C++
+    (.cpp) launches nothing and is left out."""
     h = hashlib.sha256()
     csrc = os.path.join(root, "draft_sampling_verification_head_b200", "csrc")
-    files = glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))
-    for f in sorted(files):
+    if files is None:
+        paths = glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))
+    else:
+        paths = [os.path.join(csrc, f) for f in (*files, *SHARED_HEADERS)]
+    for f in sorted(paths):
         h.update(os.path.basename(f).encode())
         h.update(_strip_comments(open(f, encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
+
+
+def kernel_hash(name: str, root: str = ROOT) -> str:
+    """csrc_hash of the sources of one profiled kernel."""
+    return csrc_hash(PROFILED_SOURCES[name], root)
 
 
 def full_stream_bytes(w) -> int:
@@ -169,7 +183,7 @@ def measured_peak():
 
 def recorded_traffic(h, name="k_cycle_tc_c3"):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source."""
+    the kernel source with hash h (kernel_hash(name) for the current one)."""
     p = os.path.join(ROOT, "profiles", f"{name}_ncu.json")
     if not os.path.exists(p):
         return None
@@ -475,7 +489,7 @@ def run_ours(args, rank, world, local_rank):
             fb = eb = draft_only_bytes(w)
             wl2 = w_l2_bytes(w, sms, greedy=True)
             kernel = "draft kernel (spec_markov_bias_sample)"
-        h = csrc_hash()
+        prof = {"cycle": "k_cycle_tc_c3", "verify": "k_verify_ee_c3"}.get(call)
         achieved = fb / (per_step_ms / 1e3) / 1e9  # GB/s over the step
         cfg = {"workload": WORKLOAD_TEXT[args.workload], "call": CALL_TEXT[call],
                "global_batch": w.B * world, "K": w.K, "V": w.V, "r": w.r,
@@ -500,7 +514,7 @@ def run_ours(args, rank, world, local_rank):
             "hbm_gbs_full_stream": achieved,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak,
-                         "traffic": (recorded_traffic(h, {"cycle": "k_cycle_tc_c3", "verify": "k_verify_ee_c3"}[call])
+                         "traffic": (recorded_traffic(kernel_hash(prof), prof)
                                      if (call in ("cycle", "verify") and args.workload == WORKLOAD) else None),
                          "peak_kind": peak_kind,
                          "bytes_per_launch": fb, "early_exit_bytes_per_launch": eb,

@@ -40,6 +40,7 @@
 //  * Every wait is bounded (spin limit); a CTA that gives up records
 //    SPEC_ERR_TIMEOUT in the workspace, the others notice and all exit.
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -535,40 +536,47 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
             // one pass: the lane's pieces p = lane + 32 u are read four at a
             // time (their shared-memory latencies overlap); stochastic rows
             // keep a running (max, sum) rescaled once per piece
-            for (int p0 = lane; p0 < npieces; p0 += 128) {
-              uint4 w4[4];
+            auto pass = [&](auto greedy_tag) {  // one code path per mode
+              constexpr bool kGreedy = decltype(greedy_tag)::value;
+              for (int p0 = lane; p0 < npieces; p0 += 128) {
+                uint4 w4[4];
   #pragma unroll
-              for (int u = 0; u < 4; ++u)
-                w4[u] = p0 + 32 * u < npieces ? sl[p0 + 32 * u] : make_uint4(0, 0, 0, 0);
+                for (int u = 0; u < 4; ++u)
+                  w4[u] = p0 + 32 * u < npieces ? sl[p0 + 32 * u] : make_uint4(0, 0, 0, 0);
   #pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const int p = p0 + 32 * u;
-                if (p >= npieces) break;
-                float x[8];
-                bf16x8(w4[u], x);
-                if (a.greedy) {
+                for (int u = 0; u < 4; ++u) {
+                  const int p = p0 + 32 * u;
+                  if (p >= npieces) break;
+                  float x[8];
+                  bf16x8(w4[u], x);
+                  if constexpr (kGreedy) {
   #pragma unroll
-                  for (int e = 0; e < 8; ++e)
-                    if (x[e] > m) {
-                      m = x[e];
-                      mi = vlo + 8 * p + e;
+                    for (int e = 0; e < 8; ++e)
+                      if (x[e] > m) {
+                        m = x[e];
+                        mi = vlo + 8 * p + e;
+                      }
+                  } else {
+                    const float m8 = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])),
+                                           fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
+                    const float mn = fmaxf(m, m8);
+                    if (mn > -INFINITY) {
+                      float sv[4];
+  #pragma unroll
+                      for (int e = 0; e < 4; ++e)
+                        sv[e] = fexp2((x[e] - mn) * k) + fexp2((x[e + 4] - mn) * k);
+                      const float s8 = (sv[0] + sv[1]) + (sv[2] + sv[3]);
+                      sm = m > -INFINITY ? fmaf(sm, fexp2((m - mn) * k), s8) : s8;
+                      m = mn;
                     }
-                } else {
-                  const float m8 = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])),
-                                         fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
-                  const float mn = fmaxf(m, m8);
-                  if (mn > -INFINITY) {
-                    float sv[4];
-  #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                      sv[e] = fexp2((x[e] - mn) * k) + fexp2((x[e + 4] - mn) * k);
-                    const float s8 = (sv[0] + sv[1]) + (sv[2] + sv[3]);
-                    sm = m > -INFINITY ? fmaf(sm, fexp2((m - mn) * k), s8) : s8;
-                    m = mn;
                   }
                 }
               }
-            }
+            };
+            if (a.greedy)
+              pass(std::true_type{});
+            else
+              pass(std::false_type{});
             __syncwarp();
             ++tcn;
             issue();  // the slot is free: the next slice is in flight while this one reduces
@@ -1301,13 +1309,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
               const int vv0 = (chunk0 + cl) * kCH + q4 * 32 + tg * SC;
               const bool full = rowok && vv0 + SC <= V;  // every token of this lane is valid
               float x[8];
+              if (full) {  // the common case without per-token checks
 #pragma unroll
-              for (int u = 0; u < NV; ++u) {
-                bf16x8(cb[u], x);
+                for (int u = 0; u < NV; ++u) {
+                  bf16x8(cb[u], x);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                  const int ee = 8 * u + e;
-                  z[ee] = (full || (rowok && vv0 + ee < V)) ? z[ee] + x[e] : -INFINITY;
+                  for (int e = 0; e < 8; ++e) z[8 * u + e] += x[e];
+                }
+              } else {
+#pragma unroll
+                for (int u = 0; u < NV; ++u) {
+                  bf16x8(cb[u], x);
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) {
+                    const int ee = 8 * u + e;
+                    z[ee] = (rowok && vv0 + ee < V) ? z[ee] + x[e] : -INFINITY;
+                  }
                 }
               }
               float m = -INFINITY;
@@ -1342,8 +1359,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
                 float sum = 0.f;
                 if (m > -INFINITY) {
                   float sv[4] = {0.f, 0.f, 0.f, 0.f};
+                  const float mk = m * k;
 #pragma unroll
-                  for (int ee = 0; ee < SC; ++ee) sv[ee & 3] += fexp2((z[ee] - m) * k);
+                  for (int ee = 0; ee < SC; ++ee) sv[ee & 3] += fexp2(fmaf(z[ee], k, -mk));
                   sum = (sv[0] + sv[1]) + (sv[2] + sv[3]);
                 }
 #pragma unroll
@@ -1508,19 +1526,46 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
               const bool any = rowok && vv0 < V;
               float r = 0.f, p = 0.f;
               float xt[8], xb[8];
+              // residual mass and target mass; a row that accepted every draft
+              // has 1 / draft sum = 0: r = p (the checks are hoisted out of the
+              // common cases; the expressions are the same in every branch)
+              if (any && vv0 + SC <= V && c.w != 0.f) {
 #pragma unroll
-              for (int u = 0; u < NV; ++u) {
-                bf16x8(ct[u], xt);
-                bf16x8(cb[u], xb);
+                for (int u = 0; u < NV; ++u) {
+                  bf16x8(ct[u], xt);
+                  bf16x8(cb[u], xb);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                  const bool ok = any && vv0 + 8 * u + e < V;
-                  // residual mass and target mass; a row that accepted every
-                  // draft has 1 / draft sum = 0: r = p
-                  const float pe = fexp2((xt[e] - c.x) * k) * c.y;
-                  const float qe = c.w != 0.f ? fexp2((z[8 * u + e] + xb[e] - c.z) * k) * c.w : 0.f;
-                  r += ok ? fmaxf(pe - qe, 0.f) : 0.f;
-                  p += ok ? pe : 0.f;
+                  for (int e = 0; e < 8; ++e) {
+                    const float pe = fexp2((xt[e] - c.x) * k) * c.y;
+                    const float qe = fexp2((z[8 * u + e] + xb[e] - c.z) * k) * c.w;
+                    r += fmaxf(pe - qe, 0.f);
+                    p += pe;
+                  }
+                }
+              } else if (any && vv0 + SC <= V) {
+#pragma unroll
+                for (int u = 0; u < NV; ++u) {
+                  bf16x8(ct[u], xt);
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) {
+                    const float pe = fexp2((xt[e] - c.x) * k) * c.y;
+                    r += pe;  // fmaxf(pe - 0, 0) = pe
+                    p += pe;
+                  }
+                }
+              } else {
+#pragma unroll
+                for (int u = 0; u < NV; ++u) {
+                  bf16x8(ct[u], xt);
+                  bf16x8(cb[u], xb);
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) {
+                    const bool ok = any && vv0 + 8 * u + e < V;
+                    const float pe = fexp2((xt[e] - c.x) * k) * c.y;
+                    const float qe = c.w != 0.f ? fexp2((z[8 * u + e] + xb[e] - c.z) * k) * c.w : 0.f;
+                    r += ok ? fmaxf(pe - qe, 0.f) : 0.f;
+                    p += ok ? pe : 0.f;
+                  }
                 }
               }
 #pragma unroll

@@ -103,6 +103,8 @@ struct ArgsTC {
   uint32_t row0;     // global index of batch row 0 (Philox counter word 1)
   int nbk;           // buckets per CTA (4 per chunk)
   int nts;           // row-slice slots per target warp (what shared memory holds)
+  int npro;          // leading positions whose target statistics the compute warps
+                     // take at the start of each job (the rest: the target warps)
 };
 
 // One record per batch row and step, written by the row's reducer.
@@ -126,7 +128,8 @@ struct CtlT {
   uint64_t wfull[kNSof<N>], wempty[kNSof<N>], dfull[2], dfree[2];
   uint64_t bready, tready, mmadone;
   uint64_t tfull[2][kTSMax];  // target row slices landed (one ring per target warp)
-  uint64_t tgo, tdone;     // target job may start / has published its partials
+  uint32_t tgo_cnt;        // target jobs released to the target warps (all jobs so far)
+  uint32_t tdone_cnt[2];   // target jobs finished by each target warp (all jobs so far)
   uint32_t tmem_slot;
   int32_t abort_local;
   int32_t prev[N];
@@ -245,6 +248,53 @@ SPEC_DEV void bf16x8(const uint4& w, float* x) {
   }
 }
 
+// Target statistics of a row slice, the same arithmetic wherever they are
+// taken.  One 16-byte piece (8 logits of tokens tok0 .. tok0 + 7) into a lane's
+// running arg-max (greedy) or (max, sum of exp2((x - max) k)), the sum
+// rescaled once per piece.
+template <bool kGreedy>
+SPEC_DEV void piece_stats(const uint4& w, int tok0, float k, float& m, float& s, int32_t& mi) {
+  float x[8];
+  bf16x8(w, x);
+  if constexpr (kGreedy) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (x[e] > m) {
+        m = x[e];
+        mi = tok0 + e;
+      }
+  } else {
+    // the piece's max in packed bf16 (exact), then one conversion
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+    const __nv_bfloat162 mx = __hmax2(__hmax2(h2[0], h2[1]), __hmax2(h2[2], h2[3]));
+    const float mn = fmaxf(m, fmaxf(__low2float(mx), __high2float(mx)));
+    if (mn > -INFINITY) {
+      const float mk = mn * k;
+      float sv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sv[e] = fexp2(fmaf(x[e], k, -mk)) + fexp2(fmaf(x[e + 4], k, -mk));
+      const float s8 = (sv[0] + sv[1]) + (sv[2] + sv[3]);
+      s = m > -INFINITY ? fmaf(s, fexp2(fmaf(m, k, -mk)), s8) : s8;
+      m = mn;
+    }
+  }
+}
+// The lanes' statistics combined over the warp (every lane gets the result).
+template <bool kGreedy>
+SPEC_DEV void warp_stats(float& m, float& s, int32_t& mi, float k) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+    if constexpr (kGreedy) {
+      const int32_t i2 = __shfl_xor_sync(0xffffffffu, mi, off);
+      amax_combine(m, mi, m2, i2);
+    } else {
+      const float s2 = __shfl_xor_sync(0xffffffffu, s, off);
+      ms_combine(m, s, m2, s2, k);
+    }
+  }
+}
+
 // Verify length K_b of row gb (cycle-major row index c * B + b): the given
 // length clamped to 1..K; or, from confidence scores, the number of leading
 // positions whose prefix survival (fp32 product of the scores of positions
@@ -326,8 +376,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
     mbar_init(&ctl->mmadone, 1);
     for (int w = 0; w < 2; ++w)
       for (int i = 0; i < kTSMax; ++i) mbar_init(&ctl->tfull[w][i], 1);
-    mbar_init(&ctl->tgo, 1);
-    mbar_init(&ctl->tdone, 2);
+    ctl->tgo_cnt = 0;
+    ctl->tdone_cnt[0] = ctl->tdone_cnt[1] = 0;
     ctl->abort_local = 0;
     fence_mbar_init();
   }
@@ -339,7 +389,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t taddr = ctl->tmem_slot;
-  if (tid == 0) mbar_arrive(&ctl->tgo);  // the first target job needs nothing else: start it now
 
   // =========================================================================
   // W producer: first the NT resident chunks (read once, by the compute warps,
@@ -463,17 +512,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
     const uint32_t bytes = (uint32_t)((vhi - vlo) * sizeof(T));
     const int npieces = (vhi - vlo) / 8;
     const uint64_t pol = policy_evict_first();
-    uint32_t tu = 0, tcn = 0, J = 0;  // copies issued, copies consumed, jobs
+    uint32_t tu = 0, tcn = 0, J = 0;  // copies issued, copies consumed, target jobs taken
     bool ok = true;
     for (int t = 0; t < njobs && ok; ++t) {
       const int g = t % a.ngroups, par = t & 1;
       const int64_t gb0 = (int64_t)(t / a.ngroups) * a.B + (int64_t)g * N;  // row 0 of the job
       const int nb_g = min(N, a.B - g * N);
-      for (int j = 0; j < K && ok; ++j, ++J) {
-        if (!mbar_wait_bounded(&ctl->tgo, J & 1, a.spin, &hdr->abort)) {
-          if (lane == 0) record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_BREADY, cta, 3000 + j);
-          ok = false;
-          break;
+      // positions below npro were taken by the compute warps at the job's start
+      for (int j = a.npro; j < K && ok; ++j, ++J) {
+        {  // wait until the compute warps release this position (bounded)
+          uint64_t it = 0;
+          while (ld_acquire_cta_smem(&ctl->tgo_cnt) <= J) {
+            if (++it >= a.spin || ((it & 63) == 0 && ld_volatile_u32(&hdr->abort))) {
+              if (lane == 0 && it >= a.spin) record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_BREADY, cta, 3000 + j);
+              ok = false;
+              break;
+            }
+            __nanosleep(64);
+          }
+          if (!ok) break;
         }
         if (a.trace && cta == 0 && t == 0 && tw == 0 && lane == 0)
           a.trace[(size_t)j * kTracePhases + 4] = globaltimer_ns();  // target job taken
@@ -547,29 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
                 for (int u = 0; u < 4; ++u) {
                   const int p = p0 + 32 * u;
                   if (p >= npieces) break;
-                  float x[8];
-                  bf16x8(w4[u], x);
-                  if constexpr (kGreedy) {
-  #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                      if (x[e] > m) {
-                        m = x[e];
-                        mi = vlo + 8 * p + e;
-                      }
-                  } else {
-                    const float m8 = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])),
-                                           fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
-                    const float mn = fmaxf(m, m8);
-                    if (mn > -INFINITY) {
-                      float sv[4];
-  #pragma unroll
-                      for (int e = 0; e < 4; ++e)
-                        sv[e] = fexp2((x[e] - mn) * k) + fexp2((x[e + 4] - mn) * k);
-                      const float s8 = (sv[0] + sv[1]) + (sv[2] + sv[3]);
-                      sm = m > -INFINITY ? fmaf(sm, fexp2((m - mn) * k), s8) : s8;
-                      m = mn;
-                    }
-                  }
+                  piece_stats<kGreedy>(w4[u], vlo + 8 * p, k, m, sm, mi);
                 }
               }
             };
@@ -580,17 +615,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
             __syncwarp();
             ++tcn;
             issue();  // the slot is free: the next slice is in flight while this one reduces
-  #pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) {
-              const float m2 = __shfl_xor_sync(FULL, m, off);
-              if (a.greedy) {
-                const int32_t i2 = __shfl_xor_sync(FULL, mi, off);
-                amax_combine(m, mi, m2, i2);
-              } else {
-                const float s2 = __shfl_xor_sync(FULL, sm, off);
-                ms_combine(m, sm, m2, s2, k);
-              }
-            }
+            if (a.greedy)
+              warp_stats<true>(m, sm, mi, k);
+            else
+              warp_stats<false>(m, sm, mi, k);
             if (lane == 0)
               a.tpart[(((int64_t)par * (K + 1) + trow) * N + n) * kMaxG + cta] =
                   a.greedy ? make_float2(m, __int_as_float(mi)) : make_float2(m, sm);
@@ -599,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         if (!ok) break;
         __threadfence();  // the partials are visible device-wide before the job is reported
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl->tdone);
+        if (lane == 0) add_release_cta_smem(&ctl->tdone_cnt[tw], 1u);
         if (a.trace && cta == 0 && t == 0 && tw == 0 && lane == 0)
           a.trace[(size_t)j * kTracePhases + 31] = globaltimer_ns();  // target job published
       }
@@ -665,6 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
       if (trace && g == 0 && jt == 0) trace[(size_t)step * kTracePhases + phase] = globaltimer_ns();
     };
 
+    mark(0, K + 1, 2);
     // ---- W^T of the resident chunks into tensor memory (once per launch).
     // Stage L (chunk L / nkb, rank block L % nkb) is read by the quartet of
     // warps L & 1: warp q4 takes tokens 32 q4 .. 32 q4 + 31 and packs two
@@ -1218,16 +1247,99 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
           if (a.draft && past) a.draft[o] = -1;
         }
       }
-      // step 0's base and target logits of this CTA's slice into L2
+      named_sync();
+      mark(g, K + 1, 0);
+      // Target statistics of positions 0 .. npro-1 (every row verifies them,
+      // and their target jobs would gate the first steps): the compute warps
+      // take them here, before the first step, with the target warps' own
+      // arithmetic.  Items (row n, target row): (n, j) for j < min(npro, K_b),
+      // and (n, K_b) when K_b <= npro (the bonus row of a row whose last
+      // verified position is among them).  A warp takes four items at a time,
+      // read straight from global memory.
+      if (a.npro > 0) {
+        // Items in a dense order: q < P nb_g is (row q % nb_g, position q / nb_g),
+        // then q - P nb_g the bonus row of that row (used when K_b <= P).  A warp
+        // takes four consecutive items at a time and reads them together.
+        auto take = [&](auto greedy_tag) {
+          constexpr bool kG = decltype(greedy_tag)::value;
+          constexpr int W = kComputeThreads / 32;
+          const int P = a.npro, slots = nb_g * (P + 1);
+          const int npieces = (vslice_hi - vslice_lo) / 8;
+          for (int q0 = warp * 4; q0 < slots; q0 += 4 * W) {
+            int nI[4], tI[4];
+            bool vI[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int q = q0 + e;
+              nI[e] = 0;
+              tI[e] = 0;
+              vI[e] = false;
+              if (q < P * nb_g) {
+                nI[e] = q % nb_g;
+                tI[e] = q / nb_g;
+                vI[e] = tI[e] < ctl->kb[nI[e]];
+              } else if (q < slots) {
+                nI[e] = q - P * nb_g;
+                tI[e] = ctl->kb[nI[e]];
+                vI[e] = tI[e] <= P;
+              }
+            }
+            if (!(vI[0] || vI[1] || vI[2] || vI[3])) continue;  // warp-uniform
+            float m[4], sm[4];
+            int32_t mi[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              m[e] = -INFINITY;
+              sm[e] = 0.f;
+              mi[e] = 0x7fffffff;
+            }
+            for (int p0 = lane; p0 < npieces; p0 += 128) {
+              uint4 w[4][4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const uint4* src = reinterpret_cast<const uint4*>(
+                    target + ((jb0 + nI[e]) * (K + 1) + tI[e]) * V + vslice_lo);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                  w[e][u] = (vI[e] && p0 + 32 * u < npieces) ? __ldcg(src + p0 + 32 * u)
+                                                             : make_uint4(0, 0, 0, 0);
+              }
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const int pp = p0 + 32 * u;
+                if (pp >= npieces) break;
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  if (vI[e]) piece_stats<kG>(w[e][u], vslice_lo + 8 * pp, k, m[e], sm[e], mi[e]);
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              if (!vI[e]) continue;  // warp-uniform
+              warp_stats<kG>(m[e], sm[e], mi[e], k);
+              if (lane == 0)
+                a.tpart[(((int64_t)par * (K + 1) + tI[e]) * N + nI[e]) * kMaxG + cta] =
+                    kG ? make_float2(m[e], __int_as_float(mi[e])) : make_float2(m[e], sm[e]);
+            }
+          }
+        };
+        if (a.greedy)
+          take(std::true_type{});
+        else
+          take(std::false_type{});
+      }
+      // step 0's base logits and the target warps' first row of this CTA's
+      // slice into L2 (after the loads above, which need the memory first)
       if (tid < nb_g) {
         const int64_t b = jb0 + tid;
         prefetch_l2_bulk(base + b * K * V + vslice_lo, slice_bytes);
-        prefetch_l2_bulk(target + b * (K + 1) * V + vslice_lo, slice_bytes);
-        if (K == 1) prefetch_l2_bulk(target + (b * (K + 1) + 1) * V + vslice_lo, slice_bytes);
+        if (a.npro < K) prefetch_l2_bulk(target + (b * (K + 1) + a.npro) * V + vslice_lo, slice_bytes);
       }
       named_sync();
-      if (tid == 0 && t > 0) mbar_arrive(&ctl->tgo);  // the target warps may take row 0 of this group
-      mark(g, K + 1, 0);
+      // the target warps may take positions npro, npro + 1 of this job
+      if (tid == 0)
+        st_release_cta_smem(&ctl->tgo_cnt, (uint32_t)(t * (K - a.npro) + min(2, K - a.npro)));
+      mark(g, K + 1, 1);
 
       for (int i = 0; i < K; ++i) {
         // ---------------- gather the Markov rows for this step
@@ -1401,13 +1513,26 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
         }
         // this CTA's target partials of row i (and row K) are out; the target
         // warps may take the next row
+        // (positions below npro were taken at the job's start); the target
+        // warps may then run up to two positions ahead
         if (tid == 0) {
-          const uint32_t J = (uint32_t)(t * K + i);  // target jobs of all earlier jobs and steps
-          if (!mbar_wait_bounded(&ctl->tdone, J & 1, a.spin, &hdr->abort)) {
-            record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_BREADY, cta, 5000 + i);
-            ctl->abort_local = 1;
+          const int KT = K - a.npro;  // target-warp positions per job
+          if (i >= a.npro) {
+            // each target warp has finished this position (a warp may be ahead)
+            const uint32_t need = (uint32_t)(t * KT + (i - a.npro) + 1);
+            uint64_t it = 0;
+            while (ld_acquire_cta_smem(&ctl->tdone_cnt[0]) < need ||
+                   ld_acquire_cta_smem(&ctl->tdone_cnt[1]) < need) {
+              if (++it >= a.spin || ((it & 63) == 0 && ld_volatile_u32(&hdr->abort))) {
+                if (it >= a.spin) record_error(hdr, SPEC_ERR_TIMEOUT, SITE_MBAR_BREADY, cta, 5000 + i);
+                ctl->abort_local = 1;
+                break;
+              }
+              __nanosleep(32);
+            }
           }
-          if (i + 1 < K) mbar_arrive(&ctl->tgo);
+          const uint32_t rel = (uint32_t)(t * KT + min(KT, max(2, i + 3 - a.npro)));
+          if (KT > 0 && rel > ctl->tgo_cnt) st_release_cta_smem(&ctl->tgo_cnt, rel);
         }
         grid_arrive();
         mark(g, i, 3);
@@ -1772,6 +1897,7 @@ cudaError_t launch_cycle_tc(const CycleLaunch& L, const CycleGeom& g, WsHeader* 
   body += rnn_p_bytes(g.N, L.r);
   a.shist = reinterpret_cast<__nv_bfloat16*>(body);
   a.nbk = g.nc * 4;
+  a.npro = std::min(2, L.K);
   a.nts = g.N == 128 ? ring_slots_tc<128>(L.r, g.nc)
         : g.N == 64 ? ring_slots_tc<64>(L.r, g.nc)
                     : (g.N == 32 ? ring_slots_tc<32>(L.r, g.nc) : ring_slots_tc<16>(L.r, g.nc));

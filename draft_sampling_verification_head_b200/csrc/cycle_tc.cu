@@ -268,15 +268,15 @@ SPEC_DEV void piece_stats(const uint4& w, int tok0, float k, float& m, float& s,
     const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
     const __nv_bfloat162 mx = __hmax2(__hmax2(h2[0], h2[1]), __hmax2(h2[2], h2[3]));
     const float mn = fmaxf(m, fmaxf(__low2float(mx), __high2float(mx)));
-    if (mn > -INFINITY) {
-      const float mk = mn * k;
-      float sv[4];
+    // without branches: while every value so far is -inf, mk = 0 and every
+    // exp2 below is exp2(-inf) = 0 (s stays 0)
+    const float mk = mn > -INFINITY ? mn * k : 0.f;
+    float sv[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sv[e] = fexp2(fmaf(x[e], k, -mk)) + fexp2(fmaf(x[e + 4], k, -mk));
-      const float s8 = (sv[0] + sv[1]) + (sv[2] + sv[3]);
-      s = m > -INFINITY ? fmaf(s, fexp2(fmaf(m, k, -mk)), s8) : s8;
-      m = mn;
-    }
+    for (int e = 0; e < 4; ++e) sv[e] = fexp2(fmaf(x[e], k, -mk)) + fexp2(fmaf(x[e + 4], k, -mk));
+    const float s8 = (sv[0] + sv[1]) + (sv[2] + sv[3]);
+    s = fmaf(s, fexp2(fmaf(m, k, -mk)), s8);
+    m = mn;
   }
 }
 // The lanes' statistics combined over the warp (every lane gets the result).
@@ -1309,15 +1309,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
                 const int pp = p0 + 32 * u;
                 if (pp >= npieces) break;
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  if (vI[e]) piece_stats<kG>(w[e][u], vslice_lo + 8 * pp, k, m[e], sm[e], mi[e]);
+                for (int e = 0; e < 4; ++e)  // unused items reduce zeros (discarded)
+                  piece_stats<kG>(w[e][u], vslice_lo + 8 * pp, k, m[e], sm[e], mi[e]);
+              }
+            }
+            // the four items' warp reductions interleaved
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float m2 = __shfl_xor_sync(FULL, m[e], off);
+                if constexpr (kG) {
+                  const int32_t i2 = __shfl_xor_sync(FULL, mi[e], off);
+                  amax_combine(m[e], mi[e], m2, i2);
+                } else {
+                  const float s2 = __shfl_xor_sync(FULL, sm[e], off);
+                  ms_combine(m[e], sm[e], m2, s2, k);
+                }
               }
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              if (!vI[e]) continue;  // warp-uniform
-              warp_stats<kG>(m[e], sm[e], mi[e], k);
-              if (lane == 0)
+              if (lane == 0 && vI[e])
                 a.tpart[(((int64_t)par * (K + 1) + tI[e]) * N + nI[e]) * kMaxG + cta] =
                     kG ? make_float2(m[e], __int_as_float(mi[e])) : make_float2(m[e], sm[e]);
             }

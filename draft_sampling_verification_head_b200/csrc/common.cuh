@@ -141,19 +141,6 @@ SPEC_DEV float load_f<__nv_bfloat16>(const __nv_bfloat16* p, int64_t i) {
 SPEC_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-// Counters in shared memory shared by the warps of one CTA (release/acquire
-// at CTA scope: what the writer stored before is visible to the reader after).
-SPEC_DEV uint32_t ld_acquire_cta_smem(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
-  return v;
-}
-SPEC_DEV void st_release_cta_smem(uint32_t* p, uint32_t v) {
-  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
-}
-SPEC_DEV void add_release_cta_smem(uint32_t* p, uint32_t v) {
-  asm volatile("red.release.cta.shared::cta.add.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
-}
 
 SPEC_DEV void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)

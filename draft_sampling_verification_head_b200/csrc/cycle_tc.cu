@@ -248,6 +248,20 @@ SPEC_DEV void bf16x8(const uint4& w, float* x) {
   }
 }
 
+// Counters in shared memory shared by the warps of one CTA (release/acquire
+// at CTA scope: what the writer stored before is visible to the reader after).
+SPEC_DEV uint32_t ld_acquire_cta_smem(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+SPEC_DEV void st_release_cta_smem(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+SPEC_DEV void add_release_cta_smem(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.cta.shared::cta.add.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+
 // Target statistics of a row slice, the same arithmetic wherever they are
 // taken.  One 16-byte piece (8 logits of tokens tok0 .. tok0 + 7) into a lane's
 // running arg-max (greedy) or (max, sum of exp2((x - max) k)), the sum

@@ -59,6 +59,11 @@ SHAPES = [
     ("ragged_v", synth.Workload("e4", B=33, K=5, V=1000 * 8 + 8, r=64, dtype="bf16", sigma=0.5, seed=114,
                                 uw_std=0.3)),
     ("k64", synth.Workload("e5", B=6, K=64, V=4096, r=64, dtype="bf16", sigma=0.1, seed=115, uw_std=0.05)),
+    # the first two positions' target statistics are taken at each job's start by
+    # the compute warps: K = 2 leaves no position to the target warps, K = 3 one
+    ("k2", synth.Workload("e6", B=20, K=2, V=6000, r=64, dtype="bf16", sigma=0.4, seed=116, uw_std=0.3)),
+    ("k3_two_groups", synth.Workload("e7", B=70, K=3, V=6000, r=64, dtype="bf16", sigma=0.4, seed=117,
+                                     uw_std=0.3)),
 ]
 
 
@@ -80,6 +85,47 @@ def test_cycle_kb_all_one():
     assert st == sd.SPEC_OK
     compare_cycle(g, ref, w.K)
     assert g["tau"].max() <= 2 and np.all(g["draft"][:, 1:] == -1)
+
+
+def test_cycle_kb_short_rows_bonus_at_the_start():
+    """Verify lengths 1 and 2 only, with K = 6: every row's bonus row is among
+    the positions whose target statistics the compute warps take first."""
+    w = SHAPES[3][1]
+    kb = np.random.default_rng(8).integers(1, 3, size=w.B).astype(np.int32)
+    for greedy in (False, True):
+        st, g, ref = _cycle_pair(w, greedy, kb=kb)
+        assert st == sd.SPEC_OK
+        f = compare_cycle(g, ref, w.K)
+        note_near(f"edge_kb12{'_greedy' if greedy else ''}", 1, w.B, f)
+        assert np.all(g["tau"] <= kb + 1)
+        assert f <= max(1, w.B // 2)
+
+
+@pytest.mark.parametrize("K", [2, 3])
+def test_decode_loop_short_blocks_two_groups(K):
+    """Chained cycles over two batch groups with K = 2 and 3 (jobs whose target
+    positions are all, or all but one, taken at the job's start)."""
+    w = synth.Workload(f"el{K}", B=70, K=K, V=6000, r=64, dtype="bf16", sigma=0.4, seed=118 + K,
+                       uw_std=0.3)
+    C = 3
+    d = synth.make_loop(w, C)
+    dd = {k: v.cuda() for k, v in d.items()}
+    for greedy in (False, True):
+        p = sd.Params(B=w.B, K=w.K, V=w.V, r=w.r, dtype=w.dtype, seed=4, cycle=9, greedy=greedy)
+        ws = sd.make_workspace(p)
+        o = sd.alloc_outputs(p, n_cycles=C)
+        nt = torch.empty(w.B, dtype=torch.int32, device="cuda")
+        sd.decode_loop(p, C, dd["base"], dd["target"], dd["U"], dd["W"], dd["last_token"],
+                       o["draft"], o["out"], o["tau"], o["p_draft"], o["q_draft"], nt, ws,
+                       conf=dd["conf"], conf_threshold=0.4)
+        assert sd.sync_status(ws) == sd.SPEC_OK
+        g = {k: _np(v) for k, v in o.items()}
+        P = oracle.Params(B=w.B, K=w.K, V=w.V, r=w.r, dtype=w.dtype, seed=4, cycle=9, greedy=greedy)
+        raw = synth.to_numpy_raw
+        ref = DL.decode_loop(P, C, raw(d["base"]), raw(d["target"]), raw(d["U"]), raw(d["W"]),
+                             d["last_token"].numpy(), conf=d["conf"].numpy(), threshold=0.4)
+        f, _ = compare_loop(g, ref, w.K)
+        note_near(f"edge_loop_k{K}{'_greedy' if greedy else ''}", 9, C * w.B, f)
 
 
 def test_decode_loop_k1():

@@ -200,7 +200,7 @@ SPEC_DEV void fence_proxy_async_smem() {
 }
 
 // ----------------------------------------------------------------------------
-// TMA (cp.async.bulk.tensor), no multicast.
+// TMA (cp.async.bulk.tensor): each CTA loads its own tiles.
 // ----------------------------------------------------------------------------
 SPEC_DEV void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

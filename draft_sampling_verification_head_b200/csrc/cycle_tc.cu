@@ -1924,7 +1924,10 @@ cudaError_t launch_cycle_tc(const CycleLaunch& L, const CycleGeom& g, WsHeader* 
   body += rnn_p_bytes(g.N, L.r);
   a.shist = reinterpret_cast<__nv_bfloat16*>(body);
   a.nbk = g.nc * 4;
-  a.npro = std::min(2, L.K);
+  // target statistics of the first positions taken by the compute warps at a
+  // job's start: two; three for long blocks of 128-row groups, whose first
+  // target jobs (128 row slices each) otherwise gate several steps
+  a.npro = std::min(g.N == 128 && L.K >= 16 ? 3 : 2, L.K);
   a.nts = g.N == 128 ? ring_slots_tc<128>(L.r, g.nc)
         : g.N == 64 ? ring_slots_tc<64>(L.r, g.nc)
                     : (g.N == 32 ? ring_slots_tc<32>(L.r, g.nc) : ring_slots_tc<16>(L.r, g.nc));

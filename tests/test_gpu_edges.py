@@ -64,6 +64,9 @@ SHAPES = [
     ("k2", synth.Workload("e6", B=20, K=2, V=6000, r=64, dtype="bf16", sigma=0.4, seed=116, uw_std=0.3)),
     ("k3_two_groups", synth.Workload("e7", B=70, K=3, V=6000, r=64, dtype="bf16", sigma=0.4, seed=117,
                                      uw_std=0.3)),
+    # 128-row groups with K >= 16 take three positions at the job's start
+    ("n128_k16", synth.Workload("e8", B=130, K=16, V=6000, r=64, dtype="bf16", sigma=0.3, seed=119,
+                                uw_std=0.3)),
 ]
 
 
@@ -85,6 +88,20 @@ def test_cycle_kb_all_one():
     assert st == sd.SPEC_OK
     compare_cycle(g, ref, w.K)
     assert g["tau"].max() <= 2 and np.all(g["draft"][:, 1:] == -1)
+
+
+def test_cycle_kb_n128_long_blocks():
+    """128-row groups, K = 16, random verify lengths 1..4: bonus rows among the
+    three positions taken at the job's start, and just after them."""
+    w = SHAPES[-1][1]
+    kb = np.random.default_rng(9).integers(1, 5, size=w.B).astype(np.int32)
+    for greedy in (False, True):
+        st, g, ref = _cycle_pair(w, greedy, kb=kb)
+        assert st == sd.SPEC_OK
+        f = compare_cycle(g, ref, w.K)
+        note_near(f"edge_n128_kb{'_greedy' if greedy else ''}", 1, w.B, f)
+        assert np.all(g["tau"] <= kb + 1)
+        assert f <= max(1, w.B // 2)
 
 
 def test_cycle_kb_short_rows_bonus_at_the_start():

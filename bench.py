@@ -381,6 +381,18 @@ def run_ours(args, rank, world, local_rank):
             raise RuntimeError("drafting for the verify inputs failed")
     if call == "rnn":
         dd["Wh"] = synth.rnn_weights(w).to(dev)
+    if call == "loop" and args.schedule:
+        # verify lengths from the host scheduler (untimed setup): the stand-in
+        # confidence scores and a stand-in steps-per-second table of a target
+        # pass over m rows -- flat up to half of the full B (K+1) rows, then
+        # falling as 1 / m (a serving engine would profile it once at start-up)
+        import numpy as np
+        full = p.B * (w.K + 1)
+        m = np.arange(full + 1, dtype=np.float64)
+        sps = 1.0 / np.maximum(m, full / 2)
+        conf = d["conf"].numpy()
+        dd["vlen"] = torch.as_tensor(
+            np.stack([sd.schedule_verify_len(conf[c], sps)[0] for c in range(C)])).to(dev)
     tau_shape = (C, p.B) if call == "loop" else (p.B,)
     tau_all = torch.zeros((max(1, args.steps),) + tau_shape, dtype=torch.int32, device=dev)
 
@@ -392,9 +404,14 @@ def run_ours(args, rank, world, local_rank):
                      o["out"], tau, o["p_draft"], o["q_draft"], ws)
         elif call == "loop":
             p.cycle = c * C
-            sd.decode_loop(p, C, dd["base"], dd["target"], dd["U"], dd["W"], dd["last_token"],
-                           o["draft"], o["out"], tau, o["p_draft"], o["q_draft"], nt, ws,
-                           conf=dd["conf"], conf_threshold=args.conf_threshold)
+            if args.schedule:
+                sd.decode_loop(p, C, dd["base"], dd["target"], dd["U"], dd["W"], dd["last_token"],
+                               o["draft"], o["out"], tau, o["p_draft"], o["q_draft"], nt, ws,
+                               verify_len=dd["vlen"])
+            else:
+                sd.decode_loop(p, C, dd["base"], dd["target"], dd["U"], dd["W"], dd["last_token"],
+                               o["draft"], o["out"], tau, o["p_draft"], o["q_draft"], nt, ws,
+                               conf=dd["conf"], conf_threshold=args.conf_threshold)
         elif call == "rnn":
             p.cycle = c
             sd.cycle_rnn(p, dd["base"], dd["target"], dd["U"], dd["W"], dd["Wh"], dd["last_token"],
@@ -446,6 +463,8 @@ def run_ours(args, rank, world, local_rank):
     ins = {"cycle": ("base", "target", "last_token"), "rnn": ("base", "target", "last_token"),
            "loop": ("base", "target", "last_token", "conf"),
            "verify": ("target", "draft_logits", "draft"), "draft": ("base", "last_token")}[call]
+    if call == "loop" and args.schedule:
+        ins = ("base", "target", "last_token", "vlen")  # the host scheduler's lengths go in
     outs = ("draft",) if call == "draft" else ("out", "tau")
     hin = {k: dd[k].cpu().pin_memory() for k in ins}
     hout = {k: torch.empty_like(o[k], device="cpu").pin_memory() for k in outs}
@@ -499,6 +518,12 @@ def run_ours(args, rank, world, local_rank):
         if call == "loop":
             cfg.update({"cycles_per_launch": C, "conf_threshold": args.conf_threshold,
                         "conf": "uniform(0.5, 1.0) per position (stand-in scores)"})
+            if args.schedule:
+                cfg.update({"conf_threshold": None,
+                            "verify_len": "spec_schedule_verify_len per cycle from the scores and a "
+                                          "stand-in steps-per-second table (flat to half of B (K+1) "
+                                          "rows, then 1/m)",
+                            "mean_verify_len": float(dd["vlen"].float().mean())})
         if call != "draft":
             cfg.update({"mean_tau": float(tau.mean()), "tau_cycles": int(tau.shape[0]),
                         "emitted_tokens_per_s": float(tau.sum()) / args.steps / (per_step_ms / 1e3)})
@@ -554,6 +579,8 @@ def main():
     ap.add_argument("--call", default="cycle", choices=sorted(CALL_TEXT),
                     help="which entry point one step runs (cycle: the headline)")
     ap.add_argument("--cycles", type=int, default=4, help="cycles per launch for --call loop")
+    ap.add_argument("--schedule", action="store_true",
+                    help="--call loop: verify lengths chosen by spec_schedule_verify_len")
     ap.add_argument("--conf-threshold", type=float, default=0.0,
                     help="prefix-survival threshold for --call loop (0: every K_b = K)")
     args = ap.parse_args()

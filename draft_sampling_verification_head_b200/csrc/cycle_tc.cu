@@ -12,8 +12,8 @@
 // Design (one launch, one CTA per SM, cooperative so all CTAs are resident):
 //  * The vocabulary is cut into 128-token chunks; CTA c owns nc consecutive
 //    chunks for the whole launch.  Batch rows are processed in groups of N
-//    (16/32/64), the tcgen05 N dimension.  Warps: 8 compute warps, a W TMA
-//    producer and the MMA issuer.
+//    (16/32/64/128), the tcgen05 N dimension.  Warps: 8 compute warps, a W TMA
+//    producer, the MMA issuer and two target warps.
 //  * The bias of a step is, per chunk, D[v, n] = W^T[v, :] . U[prev_n]^T, one
 //    tcgen05.mma kind::f16 chain (M = 128 tokens, N rows, K = r).  W^T of the
 //    CTA's first NT chunks is copied into tensor memory once per launch and
@@ -24,10 +24,15 @@
 //  * Epilogue: the accumulator tile (lane = token, column = batch row) is
 //    transposed through shared memory so that each lane holds consecutive
 //    tokens of one row; the lane adds that row's base logits (read from L2,
-//    where they were prefetched one step ahead), takes exact statistics (max,
-//    sum exp2) of each 32-token bucket, and folds in the same tokens of the
-//    row's target logits (rows still verifying; at the last draft step also
-//    target row K).  Nothing needs a second round: every statistic is exact.
+//    where they were prefetched one step ahead) and takes exact statistics
+//    (max, sum exp2) of each 32-token bucket.  Nothing needs a second round:
+//    every statistic is exact.
+//  * Target statistics (max, sum or arg-max of each target row over the
+//    CTA's slice), for rows still verifying and, at a row's last verified
+//    position, its bonus row: the first positions by the compute warps at the
+//    start of each job, the rest by the two target warps, which copy row
+//    slices into shared-memory rings and run up to two positions ahead of
+//    the draft chain.
 //  * Row n's reducer (CTA n mod G) combines the per-CTA partials in ascending
 //    token order, finds the CTA and then the bucket holding the inverse-CDF
 //    target, forms that bucket's 32 logits from the bf16 inputs with the whole
@@ -514,10 +519,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
     }
   }
   // =========================================================================
-  // Target warps: statistics of target row j (rows still verifying; at the
-  // last draft step also row K) over this CTA's slice, one job per draft step,
-  // a step ahead of the draft chain.  Each warp fetches its rows' slices with
-  // bulk copies into a private ring and reduces them from shared memory.
+  // Target warps: statistics of target row j (rows still verifying; at a
+  // row's last verified position also its bonus row K_b) over this CTA's
+  // slice, one job per position from npro on, released by the compute warps
+  // up to two positions ahead of the draft chain.  Each warp fetches its
+  // rows' slices with bulk copies into a private ring and reduces them from
+  // shared memory.
   // =========================================================================
   else if (warp >= kTargetWarp0) {
     const int tw = warp - kTargetWarp0;

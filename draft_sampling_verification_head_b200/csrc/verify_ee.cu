@@ -120,32 +120,43 @@ SPEC_DEV float piece_max(const Raw8<float>& r) {
   for (int e = 0; e < 8; ++e) m = fmaxf(m, elem(r, e));
   return m;
 }
-// sum over the piece of exp2((x - m) k), two partial sums
+// sum over the piece of exp2(x k - mk) (= exp2((x - m) k) with mk = m k),
+// two partial sums
 template <typename T>
-SPEC_DEV float piece_sumexp(const Raw8<T>& r, float m, float k) {
+SPEC_DEV float piece_sumexp(const Raw8<T>& r, float mk, float k) {
   float s0 = 0.f, s1 = 0.f;
 #pragma unroll
   for (int e = 0; e < 8; e += 2) {
-    s0 += fexp2((elem(r, e) - m) * k);
-    s1 += fexp2((elem(r, e + 1) - m) * k);
+    s0 += fexp2(fmaf(elem(r, e), k, -mk));
+    s1 += fexp2(fmaf(elem(r, e + 1), k, -mk));
   }
   return s0 + s1;
 }
-// (max, sum exp2((x - max) k)) of up to kLanePieces pieces held by this lane
+// A piece of eight -inf logits: fills the pieces a lane does not hold, so
+// that the per-lane statistics need no per-piece checks.
+template <typename T>
+SPEC_DEV Raw8<T> neg_inf_raw8() {
+  Raw8<T> r;
+  const uint32_t v = sizeof(T) == 2 ? 0xFF80FF80u : 0xFF800000u;
+#pragma unroll
+  for (int h = 0; h < (int)(sizeof(T) / 2); ++h) r.w[h] = make_uint4(v, v, v, v);
+  return r;
+}
+// (max, sum exp2((x - max) k)) of the kLanePieces pieces held by this lane
+// (pieces it does not hold are -inf), folded into (m, s)
 constexpr int kLanePieces = 4;
 template <typename T>
-SPEC_DEV void lane_ms(const Raw8<T>* x, int n, float k, float& m, float& s) {
+SPEC_DEV void lane_ms(const Raw8<T>* x, float k, float& m, float& s) {
   float mm = -INFINITY;
 #pragma unroll
-  for (int u = 0; u < kLanePieces; ++u)
-    if (u < n) mm = fmaxf(mm, piece_max(x[u]));
-  float ss = 0.f;
+  for (int u = 0; u < kLanePieces; ++u) mm = fmaxf(mm, piece_max(x[u]));
   if (mm > -INFINITY) {
+    const float mk = mm * k;
+    float ss = 0.f;
 #pragma unroll
-    for (int u = 0; u < kLanePieces; ++u)
-      if (u < n) ss += piece_sumexp(x[u], mm, k);
+    for (int u = 0; u < kLanePieces; ++u) ss += piece_sumexp(x[u], mk, k);
+    ms_combine(m, s, mm, ss, k);
   }
-  if (mm > -INFINITY) ms_combine(m, s, mm, ss, k);
 }
 
 SPEC_DEV uint64_t policy_evict_normal_v() {
@@ -555,18 +566,15 @@ __global__ void __launch_bounds__(kVThreads, 1) k_verify_ee(const __grid_constan
             for (int u0 = 0; u0 < npu; u0 += kLanePieces) {
               Raw8<T> x[kLanePieces];
               Raw8<TD> y[kLanePieces];
-              int n = 0;
 #pragma unroll
               for (int u = 0; u < kLanePieces; ++u) {
                 const int pc = 32 * (u0 + u) + lane;
-                if (u0 + u < npu && pc < np) {
-                  x[u] = load_raw8(xt + 8 * pc);
-                  y[u] = load_raw8(xd + 8 * pc);
-                  n = u + 1;
-                }
+                const bool in = u0 + u < npu && pc < np;
+                x[u] = in ? load_raw8(xt + 8 * pc) : neg_inf_raw8<T>();
+                y[u] = in ? load_raw8(xd + 8 * pc) : neg_inf_raw8<TD>();
               }
-              lane_ms(x, n, k, mt, st_);
-              lane_ms(y, n, k, md, sd_);
+              lane_ms(x, k, mt, st_);
+              lane_ms(y, k, md, sd_);
             }
             warp_ms(mt, st_, k);
             warp_ms(md, sd_, k);

@@ -101,3 +101,25 @@ def test_near_threshold_counts_flagged_and_mismatched_rows():
     tau = np.array([2, 4, 1])
     r = bench.near_threshold(ref, out, tau, K)
     assert r == {"rows_checked": 3, "flagged": 1, "mismatched_unflagged": 1}
+
+
+def test_kernel_hash_follows_code_not_comments(tmp_path):
+    """A recorded traffic figure is keyed on the profiled kernel's own source
+    and the shared headers: comments and other kernels' files do not change
+    the key, a code change in the kernel's file does."""
+    import shutil
+    src = os.path.join(ROOT, "draft_sampling_verification_head_b200", "csrc")
+    dst = tmp_path / "draft_sampling_verification_head_b200" / "csrc"
+    shutil.copytree(src, dst)
+    root = str(tmp_path)
+    h0 = {n: bench.kernel_hash(n, root) for n in bench.PROFILED_SOURCES}
+    assert h0 == {n: bench.kernel_hash(n) for n in bench.PROFILED_SOURCES}
+    cyc = dst / "cycle_tc.cu"
+    cyc.write_text(cyc.read_text() + "\n// a comment only\n/* and a block\n comment */\n")
+    assert bench.kernel_hash("k_cycle_tc_c3", root) == h0["k_cycle_tc_c3"]
+    cyc.write_text(cyc.read_text() + "\nnamespace { constexpr int kProbe = 1; }\n")
+    assert bench.kernel_hash("k_cycle_tc_c3", root) != h0["k_cycle_tc_c3"]
+    assert bench.kernel_hash("k_verify_ee_c3", root) == h0["k_verify_ee_c3"]  # another kernel's file
+    hdr = dst / "common.cuh"
+    hdr.write_text(hdr.read_text() + "\nnamespace { constexpr int kProbe2 = 2; }\n")
+    assert bench.kernel_hash("k_verify_ee_c3", root) != h0["k_verify_ee_c3"]  # a shared header

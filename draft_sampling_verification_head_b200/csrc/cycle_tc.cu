@@ -267,6 +267,27 @@ SPEC_DEV void add_release_cta_smem(uint32_t* p, uint32_t v) {
   asm volatile("red.release.cta.shared::cta.add.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
 }
 
+// Pairs of fp32 values in one 64-bit register for the packed fp32 pipe
+// (sm_100: add / fma .f32x2, each lane rounded exactly like the scalar op).
+SPEC_DEV uint64_t f2pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+SPEC_DEV void f2unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+SPEC_DEV uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+SPEC_DEV uint64_t f2add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 // Target statistics of a row slice, the same arithmetic wherever they are
 // taken.  One 16-byte piece (8 logits of tokens tok0 .. tok0 + 7) into a lane's
 // running arg-max (greedy) or (max, sum of exp2((x - max) k)), the sum
@@ -290,9 +311,15 @@ SPEC_DEV void piece_stats(const uint4& w, int tok0, float k, float& m, float& s,
     // without branches: while every value so far is -inf, mk = 0 and every
     // exp2 below is exp2(-inf) = 0 (s stays 0)
     const float mk = mn > -INFINITY ? mn * k : 0.f;
+    const uint64_t kk = f2pack(k, k), nmk = f2pack(-mk, -mk);
+    float y[8];
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) f2unpack(f2fma(f2pack(x[e], x[e + 1]), kk, nmk), y[e], y[e + 1]);
     float sv[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) sv[e] = fexp2(fmaf(x[e], k, -mk)) + fexp2(fmaf(x[e + 4], k, -mk));
+    for (int e = 0; e < 4; e += 2)
+      f2unpack(f2add(f2pack(fexp2(y[e]), fexp2(y[e + 1])), f2pack(fexp2(y[e + 4]), fexp2(y[e + 5]))),
+               sv[e], sv[e + 1]);
     const float s8 = (sv[0] + sv[1]) + (sv[2] + sv[3]);
     s = fmaf(s, fexp2(fmaf(m, k, -mk)), s8);
     m = mn;
@@ -1455,12 +1482,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
               const int vv0 = (chunk0 + cl) * kCH + q4 * 32 + tg * SC;
               const bool full = rowok && vv0 + SC <= V;  // every token of this lane is valid
               float x[8];
-              if (full) {  // the common case without per-token checks
+              if (full) {  // the common case without per-token checks (pairs: packed adds)
 #pragma unroll
                 for (int u = 0; u < NV; ++u) {
                   bf16x8(cb[u], x);
 #pragma unroll
-                  for (int e = 0; e < 8; ++e) z[8 * u + e] += x[e];
+                  for (int e = 0; e < 8; e += 2)
+                    f2unpack(f2add(f2pack(z[8 * u + e], z[8 * u + e + 1]), f2pack(x[e], x[e + 1])),
+                             z[8 * u + e], z[8 * u + e + 1]);
                 }
               } else {
 #pragma unroll
@@ -1504,10 +1533,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_cycle_tc(const __grid_constant_
                 m = fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3]));
                 float sum = 0.f;
                 if (m > -INFINITY) {
-                  float sv[4] = {0.f, 0.f, 0.f, 0.f};
+                  // four chains (element ee into chain ee % 4), kept as two packed pairs
                   const float mk = m * k;
+                  const uint64_t kk = f2pack(k, k), nmk = f2pack(-mk, -mk);
+                  uint64_t s01 = f2pack(0.f, 0.f), s23 = f2pack(0.f, 0.f);
 #pragma unroll
-                  for (int ee = 0; ee < SC; ++ee) sv[ee & 3] += fexp2(fmaf(z[ee], k, -mk));
+                  for (int ee = 0; ee < SC; ee += 4) {
+                    float y0, y1, y2, y3;
+                    f2unpack(f2fma(f2pack(z[ee], z[ee + 1]), kk, nmk), y0, y1);
+                    f2unpack(f2fma(f2pack(z[ee + 2], z[ee + 3]), kk, nmk), y2, y3);
+                    s01 = f2add(s01, f2pack(fexp2(y0), fexp2(y1)));
+                    s23 = f2add(s23, f2pack(fexp2(y2), fexp2(y3)));
+                  }
+                  float sv[4];
+                  f2unpack(s01, sv[0], sv[1]);
+                  f2unpack(s23, sv[2], sv[3]);
                   sum = (sv[0] + sv[1]) + (sv[2] + sv[3]);
                 }
 #pragma unroll
